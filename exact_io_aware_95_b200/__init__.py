@@ -1,0 +1,185 @@
+"""Python binding of the sm_100a exact-attention library (``libfa_b200.so``).
+
+Argument marshalling only: every step of the forward and backward pass runs
+in the library's CUDA kernels.  Torch provides device memory and the current
+stream.  There is no CPU or library fallback: if the compiled library is
+missing, importing any entry point raises.
+
+Layouts (see include/fa.h): dense tensors bf16 [B, N, H, d], LSE fp32
+[B, H, N]; packed tensors bf16 [total, H, d], LSE fp32 [H, total],
+cu_seqlens int32 [nseq + 1] on the device.
+"""
+from __future__ import annotations
+
+import ctypes
+import math
+import os
+from typing import Optional, Tuple
+
+import torch
+
+__all__ = ["FaError", "lib", "fwd", "bwd", "varlen_fwd", "varlen_bwd", "workspace_size", "check_device_error",
+           "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FA_ERR_WORKSPACE",
+           "EXPORTS", "LIB_PATH"]
+
+FA_OK, FA_ERR_INVALID_ARG, FA_ERR_UNSUPPORTED, FA_ERR_CUDA, FA_ERR_TIMEOUT, FA_ERR_WORKSPACE = range(6)
+
+LIB_PATH = os.path.join(os.path.dirname(os.path.abspath(__file__)), "libfa_b200.so")
+
+_P = ctypes.c_void_p
+_I = ctypes.c_int
+_F = ctypes.c_float
+_S = ctypes.c_size_t
+
+# name -> (restype, argtypes); mirrors include/fa.h
+EXPORTS = {
+    "fa_fwd": (_I, [_P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_varlen_fwd": (_I, [_P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_varlen_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_status_string": (ctypes.c_char_p, [_I]),
+    "fa_get_device_error": (_I, [_P]),
+}
+
+
+class FaError(RuntimeError):
+    def __init__(self, status: int, where: str):
+        self.status = status
+        super().__init__(f"{where}: {status_string(status)} (status {status})")
+
+
+_lib = None
+
+
+def lib(path: Optional[str] = None):
+    """Load the compiled library (once).  Raises if it has not been built."""
+    global _lib
+    if _lib is not None and path is None:
+        return _lib
+    p = path or LIB_PATH
+    if not os.path.exists(p):
+        raise ImportError(f"CUDA library {p} is missing; build it with exact_io_aware_95_b200.build.build()")
+    L = ctypes.CDLL(p)
+    for name, (res, args) in EXPORTS.items():
+        f = getattr(L, name)
+        f.restype = res
+        f.argtypes = args
+    if path is None:
+        _lib = L
+    return L
+
+
+def status_string(s: int) -> str:
+    return lib().fa_status_string(int(s)).decode()
+
+
+def _check(status: int, where: str):
+    if status != FA_OK:
+        raise FaError(status, where)
+
+
+def _stream_ptr(t: torch.Tensor) -> int:
+    return torch.cuda.current_stream(t.device).cuda_stream
+
+
+def _need(t: torch.Tensor, name: str, dtype, ndim: int):
+    if not isinstance(t, torch.Tensor):
+        raise TypeError(f"{name} must be a torch.Tensor")
+    if t.dtype != dtype:
+        raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
+    if t.dim() != ndim:
+        raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
+    if not t.is_cuda:
+        raise ValueError(f"{name} must be on a CUDA device")
+    if not t.is_contiguous():
+        raise ValueError(f"{name} must be contiguous")
+
+
+def _scale(scale: Optional[float], d: int) -> float:
+    return 1.0 / math.sqrt(d) if scale is None else float(scale)
+
+
+def workspace_size(B: int, N: int, H: int, d: int) -> int:
+    return int(lib().fa_bwd_workspace_size(B, N, H, d))
+
+
+def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False, scale: Optional[float] = None,
+        out: Optional[torch.Tensor] = None, lse: Optional[torch.Tensor] = None) -> Tuple[torch.Tensor, torch.Tensor]:
+    """O, LSE = attention(q, k, v) for dense [B, N, H, d] bf16 inputs."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, N, H, d]")
+    B, N, H, d = q.shape
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need(o, "out", torch.bfloat16, 4)
+    _need(l, "lse", torch.float32, 3)
+    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, N, H, d,
+                      _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_fwd")
+    return o, l
+
+
+def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
+        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None):
+    """dQ, dK, dV for dense [B, N, H, d] inputs (o, lse from fwd)."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, n, torch.bfloat16, 4)
+    _need(lse, "lse", torch.float32, 3)
+    B, N, H, d = q.shape
+    ws_need = workspace_size(B, N, H, d)
+    ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                      B, N, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_bwd")
+    return dq, dk, dv
+
+
+def varlen_fwd(q, k, v, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = False,
+               scale: Optional[float] = None, out=None, lse=None):
+    """Packed forward: q, k, v [total, H, d]; returns O [total, H, d], LSE [H, total]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    total, H, d = q.shape
+    nseq = cu_seqlens.numel() - 1
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((H, total), dtype=torch.float32, device=q.device) if lse is None else lse
+    st = lib().fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                             cu_seqlens.data_ptr(), nseq, total, int(max_seqlen), H, d, _scale(scale, d),
+                             int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_varlen_fwd")
+    return o, l
+
+
+def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = False,
+               scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None):
+    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need(t, n, torch.bfloat16, 3)
+    _need(lse, "lse", torch.float32, 2)
+    _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
+    total, H, d = q.shape
+    nseq = cu_seqlens.numel() - 1
+    ws_need = workspace_size(1, total, H, d)
+    ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
+    dq = torch.empty_like(q) if dq is None else dq
+    dk = torch.empty_like(k) if dk is None else dk
+    dv = torch.empty_like(v) if dv is None else dv
+    st = lib().fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                             ws.numel() * ws.element_size(), cu_seqlens.data_ptr(), nseq, total, int(max_seqlen),
+                             H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_varlen_bwd")
+    return dq, dk, dv
+
+
+def check_device_error(stream: Optional[torch.cuda.Stream] = None):
+    """Synchronise the stream and raise if a kernel gave up on a bounded wait."""
+    s = (stream or torch.cuda.current_stream()).cuda_stream
+    _check(lib().fa_get_device_error(s), "fa_get_device_error")

@@ -1,0 +1,335 @@
+// C-ABI entry points of the exact-attention library (declared in include/fa.h):
+// host-side validation, TMA tensor-map construction, template dispatch and
+// launch.  No device memory is allocated here; no compute happens on the host.
+#include <cuda.h>
+#include <cuda_runtime.h>
+
+#include <cmath>
+#include <cstdint>
+#include <mutex>
+
+#include "fa.h"
+
+// Forward variant: P through tensor memory (1) or through shared memory (0).
+#ifndef FA_FWD_P_IN_TMEM
+#define FA_FWD_P_IN_TMEM 1
+#endif
+#include "fa_bwd.cuh"
+#include "fa_fwd.cuh"
+
+namespace {
+
+using EncodeTiledFn = CUresult (*)(CUtensorMap*, CUtensorMapDataType, cuuint32_t, void*, const cuuint64_t*,
+                                   const cuuint64_t*, const cuuint32_t*, const cuuint32_t*, CUtensorMapInterleave,
+                                   CUtensorMapSwizzle, CUtensorMapL2promotion, CUtensorMapFloatOOBfill);
+
+std::mutex g_mu;
+
+EncodeTiledFn encode_fn() {
+  static EncodeTiledFn fn = nullptr;
+  static bool tried = false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<EncodeTiledFn>(ptr);
+  }
+  return fn;
+}
+
+constexpr int kMaxDevices = 64;
+
+// Per-device: compute capability check result and the opt-in shared-memory
+// attribute of each kernel instantiation (set once per device).
+struct DeviceState {
+  int checked = 0;  // 0 unknown, 1 sm_100, -1 other
+};
+DeviceState g_dev[kMaxDevices];
+
+fa_status current_device(int* dev) {
+  if (cudaGetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  if (*dev < 0 || *dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  std::lock_guard<std::mutex> lk(g_mu);
+  DeviceState& st = g_dev[*dev];
+  if (st.checked == 0) {
+    int major = 0, minor = 0;
+    if (cudaDeviceGetAttribute(&major, cudaDevAttrComputeCapabilityMajor, *dev) != cudaSuccess ||
+        cudaDeviceGetAttribute(&minor, cudaDevAttrComputeCapabilityMinor, *dev) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    st.checked = (major == 10 && minor == 0) ? 1 : -1;
+  }
+  return st.checked == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
+}
+
+// Set the dynamic shared-memory limit of `kern` once per device.
+template <typename K>
+fa_status ensure_smem(K kern, int dev, int bytes, bool* done_flags) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!done_flags[dev]) {
+    if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    done_flags[dev] = true;
+  }
+  return FA_OK;
+}
+
+bool aligned16(const void* p) { return (reinterpret_cast<uintptr_t>(p) & 15u) == 0; }
+
+// Tensor map over a bf16 array laid out [outer, rows, H, d] (d innermost),
+// read in boxes of 64 (d) x 1 (head) x box_rows (rows) with 128-byte swizzle.
+fa_status make_map_bf16(CUtensorMap* m, const void* base, int d, int H, int64_t rows, int64_t outer,
+                        int box_rows) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t dims[4] = {(cuuint64_t)d, (cuuint64_t)H, (cuuint64_t)rows, (cuuint64_t)outer};
+  cuuint64_t strides[3] = {(cuuint64_t)d * 2, (cuuint64_t)H * d * 2, (cuuint64_t)rows * H * d * 2};
+  cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+fa_status launch_status() {
+  cudaError_t e = cudaGetLastError();
+  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+}
+
+constexpr float kLog2e = 1.4426950408889634f;
+
+// ------------------------------------------------------------------ forward
+template <int D, bool CAUSAL, bool VARLEN>
+fa_status launch_fwd(int dev, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
+                     const fa::FwdParams& p, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  constexpr bool PTM = FA_FWD_P_IN_TMEM;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, VARLEN, PTM>;
+  constexpr int smem = fa::FwdCfg<D, PTM>::SMEM_BYTES;
+  fa_status st = ensure_smem(kern, dev, smem, done);
+  if (st != FA_OK) return st;
+  const int64_t grid = static_cast<int64_t>(p.npairs) * p.B * p.H;
+  if (grid <= 0 || grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
+  kern<<<static_cast<unsigned>(grid), fa::FwdCfg<D, PTM>::THREADS, smem, s>>>(q, k, v, p);
+  return launch_status();
+}
+
+template <int D>
+fa_status dispatch_fwd(int dev, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
+                       const CUtensorMap& v, const fa::FwdParams& p, cudaStream_t s) {
+  if (varlen) return causal ? launch_fwd<D, true, true>(dev, q, k, v, p, s) : launch_fwd<D, false, true>(dev, q, k, v, p, s);
+  return causal ? launch_fwd<D, true, false>(dev, q, k, v, p, s) : launch_fwd<D, false, false>(dev, q, k, v, p, s);
+}
+
+fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu, int B,
+                     int N, int total, int H, int d, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || total < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const bool varlen = cu != nullptr;
+  const int64_t rows = varlen ? total : N;
+  const int64_t outer = varlen ? 1 : B;
+  if (rows * outer * H * d > (int64_t(1) << 40)) return FA_ERR_INVALID_ARG;
+  int dev;
+  fa_status st = current_device(&dev);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv;
+  if ((st = make_map_bf16(&mq, q, d, H, rows, outer, 128)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mk, k, d, H, rows, outer, 128)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mv, v, d, H, rows, outer, 128)) != FA_OK) return st;
+  fa::FwdParams p;
+  p.o = o;
+  p.lse = lse;
+  p.cu_seqlens = cu;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.total = varlen ? total : N;
+  p.npairs = (N + 255) / 256;
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? dispatch_fwd<64>(dev, causal, varlen, mq, mk, mv, p, s)
+                 : dispatch_fwd<128>(dev, causal, varlen, mq, mk, mv, p, s);
+}
+
+// ----------------------------------------------------------------- backward
+size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
+
+size_t ws_bytes_for(int64_t rows, int H, int d) {
+  return align256(static_cast<size_t>(rows) * H * d * sizeof(float)) + align256(static_cast<size_t>(rows) * H * sizeof(float));
+}
+
+template <int D, bool CAUSAL, bool VARLEN>
+fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                     const CUtensorMap& mdo, const fa::BwdParams& p, cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL, VARLEN>;
+  constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
+  fa_status st = ensure_smem(kern, dev, smem, done);
+  if (st != FA_OK) return st;
+  // 1) D = rowsum(dO * O) and zeroed dQ accumulator
+  {
+    const int64_t rows = static_cast<int64_t>(p.rows) * p.H;  // one warp per (token, head)
+    const int64_t blocks = (rows + 7) / 8;
+    if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    if ((st = launch_status()) != FA_OK) return st;
+  }
+  // 2) fused recompute + dK, dV, dQ accumulation, one CTA per 128-key tile
+  {
+    const int64_t grid = static_cast<int64_t>(p.nkvtiles) * p.B * p.H;
+    if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    kern<<<static_cast<unsigned>(grid), fa::BwdCfg<D>::THREADS, smem, s>>>(mq, mk, mv, mdo, p);
+    if ((st = launch_status()) != FA_OK) return st;
+  }
+  // 3) dQ = bf16(scale * dQ accumulator)
+  {
+    const int64_t n8 = static_cast<int64_t>(p.rows) * p.H * D / 8;
+    const int64_t blocks = (n8 + 255) / 256;
+    if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    fa::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p.dq_acc, p.dq, n8, p.scale);
+    if ((st = launch_status()) != FA_OK) return st;
+  }
+  return FA_OK;
+}
+
+template <int D>
+fa_status dispatch_bwd(int dev, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
+                       const CUtensorMap& v, const CUtensorMap& d_o, const fa::BwdParams& p, cudaStream_t s) {
+  if (varlen)
+    return causal ? launch_bwd<D, true, true>(dev, q, k, v, d_o, p, s) : launch_bwd<D, false, true>(dev, q, k, v, d_o, p, s);
+  return causal ? launch_bwd<D, true, false>(dev, q, k, v, d_o, p, s) : launch_bwd<D, false, false>(dev, q, k, v, d_o, p, s);
+}
+
+fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                     void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const int* cu, int B, int N, int total,
+                     int H, int d, float scale, int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !ws) return FA_ERR_INVALID_ARG;
+  const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, ws};
+  for (const void* ptr : ptrs)
+    if (!aligned16(ptr)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(ws) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1 || total < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  const bool varlen = cu != nullptr;
+  const int64_t rows = varlen ? total : N;
+  const int64_t outer = varlen ? 1 : B;
+  if (rows * outer * H * d > (int64_t(1) << 40)) return FA_ERR_INVALID_ARG;
+  const size_t need = ws_bytes_for(rows * outer, H, d);
+  if (ws_bytes < need) return FA_ERR_WORKSPACE;
+  int dev;
+  fa_status st = current_device(&dev);
+  if (st != FA_OK) return st;
+  CUtensorMap mq, mk, mv, mdo;
+  if ((st = make_map_bf16(&mq, q, d, H, rows, outer, 128)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mk, k, d, H, rows, outer, 128)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mv, v, d, H, rows, outer, 128)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mdo, dO, d, H, rows, outer, 128)) != FA_OK) return st;
+  fa::BwdParams p;
+  p.o = o;
+  p.dout = dO;
+  p.lse = lse;
+  p.dq = dq;
+  p.dk = dk;
+  p.dv = dv;
+  p.dq_acc = static_cast<float*>(ws);
+  p.dvec = reinterpret_cast<float*>(static_cast<char*>(ws) + align256(static_cast<size_t>(rows * outer) * H * d * sizeof(float)));
+  p.cu_seqlens = cu;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.total = varlen ? total : N;
+  p.rows = static_cast<int>(rows * outer);
+  p.nkvtiles = (N + 127) / 128;
+  p.scale = scale;
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  return d == 64 ? dispatch_bwd<64>(dev, causal, varlen, mq, mk, mv, mdo, p, s)
+                 : dispatch_bwd<128>(dev, causal, varlen, mq, mk, mv, mdo, p, s);
+}
+
+bool valid_cu(const int* cu, int nseq, int total, int max_seqlen) {
+  return cu && nseq >= 1 && total >= 1 && max_seqlen >= 1;
+}
+
+}  // namespace
+
+extern "C" {
+
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int d,
+                 float scale, int causal, void* stream) {
+  return fwd_common(q, k, v, o, lse, nullptr, B, N, N, H, d, scale, causal, stream);
+}
+
+fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
+                        int nseq, int total, int max_seqlen, int H, int d, float scale, int causal, void* stream) {
+  if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  return fwd_common(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, d, scale, causal, stream);
+}
+
+size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || (d != 64 && d != 128)) return 0;
+  return ws_bytes_for(static_cast<int64_t>(B) * N, H, d);
+}
+
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                 void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int N, int H, int d,
+                 float scale, int causal, void* stream) {
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, N, H, d, scale, causal,
+                    stream);
+}
+
+fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
+                        void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, const int* cu_seqlens,
+                        int nseq, int total, int max_seqlen, int H, int d, float scale, int causal, void* stream) {
+  if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total, H, d,
+                    scale, causal, stream);
+}
+
+const char* fa_status_string(fa_status s) {
+  switch (s) {
+    case FA_OK: return "ok";
+    case FA_ERR_INVALID_ARG: return "invalid argument (null/misaligned pointer or bad size)";
+    case FA_ERR_UNSUPPORTED: return "unsupported (head dim must be 64 or 128; device must be sm_100)";
+    case FA_ERR_CUDA: return "CUDA error";
+    case FA_ERR_TIMEOUT: return "device pipeline wait timed out";
+    case FA_ERR_WORKSPACE: return "workspace too small";
+  }
+  return "unknown status";
+}
+
+fa_status fa_get_device_error(void* stream) {
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (cudaStreamSynchronize(s) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  unsigned int word = 0, zero = 0;
+  if (cudaMemcpyFromSymbol(&word, fa::g_fa_error_word, sizeof(word)) != cudaSuccess ||
+      cudaMemcpyToSymbol(fa::g_fa_error_word, &zero, sizeof(zero)) != cudaSuccess) {
+    cudaGetLastError();
+    return FA_ERR_CUDA;
+  }
+  return word ? FA_ERR_TIMEOUT : FA_OK;
+}
+
+}  // extern "C"

@@ -1,0 +1,495 @@
+// Exact-attention backward for sm_100a: recompute instead of store.
+//
+// Nothing of size N x N was kept by the forward pass; only O and the per-row
+// logsumexp.  The backward pass rebuilds each 128 x 128 block of P from Q, K
+// and the logsumexp and uses it at once ("FlashAttention: Fast and
+// Memory-Efficient Exact Attention with IO-Awareness", section "Recalcular en
+// vez de guardar"; "FlashAttention" (freenetmedia.pl), section "Jak dzialaja
+// FlashAttention?").  Three kernels:
+//
+//   1. preprocess   D_i = sum_c dO_ic O_ic (fp32), and the fp32 dQ accumulator
+//                   is zeroed.  D_i equals P_i . dP_i, the row term of the
+//                   softmax Jacobian product.
+//   2. main         one CTA per (128-key tile j, batch entry or sequence, head);
+//                   K_j and V_j stay in shared memory while the CTA loops over
+//                   the query tiles i that can see them:
+//                     S^T  = K_j Q_i^T                 (tcgen05, tensor memory)
+//                     P^T  = exp2(S^T c - LSE_i log2 e) -> bf16 in tensor memory
+//                     dP^T = V_j dO_i^T                (tcgen05)
+//                     dV  += P^T dO_i                  (tcgen05, A from tensor memory)
+//                     dS^T = P^T (dP^T - D_i)          -> bf16 in shared memory
+//                     dK  += dS^T Q_i                  (tcgen05)
+//                     dQ_i = dS K_j                    (tcgen05, dS^T read transposed)
+//                   and dQ_i is added into the fp32 accumulator with vector
+//                   atomics.  dK (times scale) and dV are stored once.
+//   3. dq_convert   dQ = bf16(scale * accumulator).
+//
+// Working with S^T instead of S puts one key per tensor-memory lane, so each
+// thread owns one row of P^T and dS^T: exactly the A operands of the dV and dK
+// products.  The dQ product reads the same dS^T buffer through an MN-major
+// descriptor, so dS is written once.
+//
+// Warp roles of the main kernel (320 threads):
+//   warps 0-3  P^T and dS^T (thread t = key row t), final dK/dV stores
+//   warps 4-7  dQ_i drain: tensor memory -> fp32 atomics (thread t = query row t)
+//   warp  8    TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring
+//   warp  9    tensor-memory allocator and the single MMA-issuing thread
+#pragma once
+#include "sm100_ptx.cuh"
+
+namespace fa {
+
+struct BwdParams {
+  const void* o;
+  const void* dout;
+  const float* lse;
+  void* dq;
+  void* dk;
+  void* dv;
+  float* dq_acc;  // fp32, same [rows, H, d] layout as dq
+  float* dvec;    // fp32 D, same indexing as lse
+  const int* cu_seqlens;
+  int B;         // dense: batch; packed: number of sequences
+  int N;         // dense: sequence length; packed: max sequence length
+  int H;
+  int total;     // packed: total tokens; dense: N
+  int rows;      // B*N (dense) or total (packed)
+  int nkvtiles;  // ceil(N / 128)
+  float scale;
+  float scale_log2;
+};
+
+// ------------------------------------------------------------------ preprocess
+// One warp per (token, head) row.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams p) {
+  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int lane = threadIdx.x & 31;
+  const int64_t nrows = static_cast<int64_t>(p.rows) * p.H;
+  if (w >= nrows) return;
+  const int64_t tok = w / p.H;
+  const int h = static_cast<int>(w % p.H);
+  const size_t base = static_cast<size_t>(w) * D;  // [rows, H, D] element offset
+  constexpr int PER = D / 32;                      // elements per lane (2 or 4)
+  const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(p.o) + base + lane * PER;
+  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(p.dout) + base + lane * PER;
+  float acc = 0.f;
+  if (PER == 4) {
+    const uint2 ov = *reinterpret_cast<const uint2*>(o);
+    const uint2 gv = *reinterpret_cast<const uint2*>(g);
+    acc = bf16lo_to_f32(ov.x) * bf16lo_to_f32(gv.x) + bf16hi_to_f32(ov.x) * bf16hi_to_f32(gv.x) +
+          bf16lo_to_f32(ov.y) * bf16lo_to_f32(gv.y) + bf16hi_to_f32(ov.y) * bf16hi_to_f32(gv.y);
+  } else {
+    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o);
+    const uint32_t gv = *reinterpret_cast<const uint32_t*>(g);
+    acc = bf16lo_to_f32(ov) * bf16lo_to_f32(gv) + bf16hi_to_f32(ov) * bf16hi_to_f32(gv);
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+  float* acc_row = p.dq_acc + base + lane * PER;
+#pragma unroll
+  for (int i = 0; i < PER; ++i) acc_row[i] = 0.f;
+  if (lane == 0) {
+    size_t li;
+    if (p.cu_seqlens) {
+      li = static_cast<size_t>(h) * p.total + tok;
+    } else {
+      const int64_t b = tok / p.N, n = tok % p.N;
+      li = (static_cast<size_t>(b) * p.H + h) * p.N + n;
+    }
+    p.dvec[li] = acc;
+  }
+}
+
+// ------------------------------------------------------------------ dQ convert
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc, void* dq, int64_t n8,
+                                                                 float scale) {
+  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  if (i >= n8) return;
+  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
+  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
+  uint4 r;
+  r.x = pack_bf16x2(a.x * scale, a.y * scale);
+  r.y = pack_bf16x2(a.z * scale, a.w * scale);
+  r.z = pack_bf16x2(b.x * scale, b.y * scale);
+  r.w = pack_bf16x2(b.z * scale, b.w * scale);
+  reinterpret_cast<uint4*>(dq)[i] = r;
+}
+
+// ------------------------------------------------------------------ main kernel
+template <int D>
+struct BwdCfg {
+  static constexpr int TILE_BYTES = 128 * D * 2;
+  static constexpr int NCHUNK = D / 64;
+  static constexpr int NSTAGE = 2;
+  static constexpr int DS_BYTES = 128 * 128 * 2;
+  static constexpr int OFF_K = 0;
+  static constexpr int OFF_V = OFF_K + TILE_BYTES;
+  static constexpr int OFF_Q = OFF_V + TILE_BYTES;                 // NSTAGE tiles
+  static constexpr int OFF_DO = OFF_Q + NSTAGE * TILE_BYTES;       // NSTAGE tiles
+  static constexpr int OFF_DS = OFF_DO + NSTAGE * TILE_BYTES;
+  static constexpr int OFF_LSE = OFF_DS + DS_BYTES;                // 128 fp32
+  static constexpr int OFF_DV = OFF_LSE + 512;                     // 128 fp32
+  static constexpr int OFF_BAR = OFF_DV + 512;
+  static constexpr int BAR_KV = 0;
+  static constexpr int BAR_QDO_FULL = 1;
+  static constexpr int BAR_QDO_EMPTY = BAR_QDO_FULL + NSTAGE;
+  static constexpr int BAR_S = BAR_QDO_EMPTY + NSTAGE;
+  static constexpr int BAR_DP = BAR_S + 1;
+  static constexpr int BAR_P = BAR_DP + 1;
+  static constexpr int BAR_DS = BAR_P + 1;
+  static constexpr int BAR_DS_EMPTY = BAR_DS + 1;
+  static constexpr int BAR_DQ_FULL = BAR_DS_EMPTY + 1;
+  static constexpr int BAR_DQ_EMPTY = BAR_DQ_FULL + 1;
+  static constexpr int BAR_ACC = BAR_DQ_EMPTY + 1;
+  static constexpr int BAR_DRAIN = BAR_ACC + 1;
+  static constexpr int NBAR = BAR_DRAIN + 1;
+  static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
+  static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
+  // tensor memory: S^T (P^T packed into its first 64 columns) | dP^T | dK | dV  [| dQ]
+  static constexpr int TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
+  static constexpr bool DQ_ALIASES_DP = (256 + 2 * D + D) > 512;
+  static constexpr int TM_DQ = DQ_ALIASES_DP ? TM_DP : 256 + 2 * D;
+  static constexpr int TMEM_COLS = 512;
+  static constexpr int THREADS = 320;
+  static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+};
+
+template <int D, bool CAUSAL, bool VARLEN>
+__global__ void __launch_bounds__(320, 1)
+    fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
+                  const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
+                  const BwdParams p) {
+  using C = BwdCfg<D>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  const uint32_t sbase = smem_u32(smem);
+  const int warp = threadIdx.x >> 5;
+  const int lane = threadIdx.x & 31;
+
+  // ---- work item: (key tile j, batch entry or sequence, head); longest key tiles first
+  int x = blockIdx.x;
+  const int h = x % p.H;
+  x /= p.H;
+  const int b = x % p.B;
+  x /= p.B;
+  const int j = x;
+  int L, tok0, bcoord;
+  if (VARLEN) {
+    tok0 = p.cu_seqlens[b];
+    L = p.cu_seqlens[b + 1] - tok0;
+    bcoord = 0;
+    if (tok0 < 0 || L < 0 || tok0 + L > p.total || L > p.N) {  // offsets inconsistent with total / max_seqlen
+      if (threadIdx.x == 0) atomicOr(&g_fa_error_word, FA_DEVERR_BOUNDS);
+      return;
+    }
+  } else {
+    tok0 = 0;
+    L = p.N;
+    bcoord = b;
+  }
+  const int k0 = 128 * j;
+  if (k0 >= L) return;
+  const int nq = (L + 127) >> 7;
+  const int i_begin = CAUSAL ? j : 0;
+  const int niter = nq - i_begin;
+
+  auto bar = [&](int i) -> uint32_t { return sbase + C::OFF_BAR + 8u * i; };
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(smem + C::OFF_MISC + 4);
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(smem + C::OFF_MISC);
+
+  if (threadIdx.x == 0) {
+    mbar_init(bar(C::BAR_KV), 1);
+    for (int s = 0; s < C::NSTAGE; ++s) {
+      mbar_init(bar(C::BAR_QDO_FULL + s), 1);
+      mbar_init(bar(C::BAR_QDO_EMPTY + s), 1);
+    }
+    mbar_init(bar(C::BAR_S), 1);
+    mbar_init(bar(C::BAR_DP), 1);
+    mbar_init(bar(C::BAR_P), 128);
+    mbar_init(bar(C::BAR_DS), 128);
+    mbar_init(bar(C::BAR_DS_EMPTY), 1);
+    mbar_init(bar(C::BAR_DQ_FULL), 1);
+    mbar_init(bar(C::BAR_DQ_EMPTY), 128);
+    mbar_init(bar(C::BAR_ACC), 1);
+    mbar_init(bar(C::BAR_DRAIN), 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 9) {
+    tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem = *tmem_slot;
+
+  if (warp == 8) {
+    // ------------------------------------------------------------ producer
+    if (lane == 0) {
+      tma_prefetch_desc(&tmQ);
+      tma_prefetch_desc(&tmK);
+      tma_prefetch_desc(&tmV);
+      tma_prefetch_desc(&tmdO);
+      mbar_arrive_expect_tx(bar(C::BAR_KV), 2 * C::TILE_BYTES);
+      for (int c = 0; c < C::NCHUNK; ++c) {
+        tma_load_4d(sbase + C::OFF_K + c * 16384, &tmK, bar(C::BAR_KV), c * 64, h, tok0 + k0, bcoord);
+        tma_load_4d(sbase + C::OFF_V + c * 16384, &tmV, bar(C::BAR_KV), c * 64, h, tok0 + k0, bcoord);
+      }
+      int issued = 0;
+      for (int it = 0; it < niter; ++it) {
+        const int st = it % C::NSTAGE;
+        const uint32_t ph = (it / C::NSTAGE) & 1;
+        if (!mbar_wait(bar(C::BAR_QDO_EMPTY + st), ph ^ 1u, abort_flag)) break;
+        const int q0 = 128 * (i_begin + it);
+        mbar_arrive_expect_tx(bar(C::BAR_QDO_FULL + st), 2 * C::TILE_BYTES);
+        for (int c = 0; c < C::NCHUNK; ++c) {
+          tma_load_4d(sbase + C::OFF_Q + st * C::TILE_BYTES + c * 16384, &tmQ, bar(C::BAR_QDO_FULL + st), c * 64, h,
+                      tok0 + q0, bcoord);
+          tma_load_4d(sbase + C::OFF_DO + st * C::TILE_BYTES + c * 16384, &tmdO, bar(C::BAR_QDO_FULL + st), c * 64,
+                      h, tok0 + q0, bcoord);
+        }
+        ++issued;
+      }
+      if (*abort_flag) {
+        mbar_wait_drain(bar(C::BAR_KV), 0);
+        for (int i = 0; i < C::NSTAGE && i < issued; ++i) {
+          const int n = issued - 1 - i;
+          mbar_wait_drain(bar(C::BAR_QDO_FULL + n % C::NSTAGE), (n / C::NSTAGE) & 1);
+        }
+      }
+    }
+    __syncwarp();
+  } else if (warp == 9) {
+    // ------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t kIdSq = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
+      constexpr uint32_t kIdDV = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK
+      constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, true, true);      // dQ: A = dS (MN-major view)
+      bool ok = mbar_wait(bar(C::BAR_KV), 0, abort_flag);
+      if (ok) tc_fence_after();
+      for (int it = 0; ok && it < niter; ++it) {
+        const int st = it % C::NSTAGE;
+        const uint32_t ph = (it / C::NSTAGE) & 1;
+        const uint32_t par = it & 1;
+        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
+        const uint32_t sdO = sbase + C::OFF_DO + st * C::TILE_BYTES;
+        if (!(ok = mbar_wait(bar(C::BAR_QDO_FULL + st), ph, abort_flag))) break;
+        tc_fence_after();
+        // S^T = K Q^T
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S, sdesc_sw128(sbase + C::OFF_K + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
+                  kIdSq, kk > 0);
+        }
+        umma_commit(bar(C::BAR_S));
+        // dP^T = V dO^T  (its columns may hold the previous dQ_i: wait until drained)
+        if (C::DQ_ALIASES_DP && it > 0) {
+          if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP, sdesc_sw128(sbase + C::OFF_V + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024),
+                  kIdSq, kk > 0);
+        }
+        umma_commit(bar(C::BAR_DP));
+        // dV += P^T dO   (A = P^T packed bf16 in tensor memory)
+        if (!(ok = mbar_wait(bar(C::BAR_P), par, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdDV,
+                  (it > 0 || kk > 0));
+        // dK += dS^T Q ;  dQ_i = dS K
+        if (!(ok = mbar_wait(bar(C::BAR_DS), par, abort_flag))) break;
+        tc_fence_after();
+        const uint32_t sDS = sbase + C::OFF_DS;
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + C::TM_DK, sdesc_sw128(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
+                  sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdDV, (it > 0 || kk > 0));
+        if (!C::DQ_ALIASES_DP && it > 0) {
+          if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
+          tc_fence_after();
+        }
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ss(tmem + C::TM_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
+                  sdesc_sw128(sbase + C::OFF_K + kk * 2048, 16384, 1024), kIdDQ, kk > 0);
+        umma_commit(bar(C::BAR_QDO_EMPTY + st));
+        umma_commit(bar(C::BAR_DS_EMPTY));
+        umma_commit(bar(C::BAR_DQ_FULL));
+      }
+      if (ok) umma_commit(bar(C::BAR_ACC));
+      if (*abort_flag) {
+        umma_commit(bar(C::BAR_DRAIN));
+        mbar_wait_drain(bar(C::BAR_DRAIN), 0);
+      }
+    }
+    __syncwarp();
+  } else if (warp < 4) {
+    // ------------------------------------------------------------ P^T and dS^T
+    const int t = threadIdx.x;  // key row within the tile == tensor-memory lane
+    const int key = k0 + t;
+    const bool key_ok = key < L;
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    float* sLSE = reinterpret_cast<float*>(smem + C::OFF_LSE);
+    float* sDv = reinterpret_cast<float*>(smem + C::OFF_DV);
+    const float c = p.scale_log2;
+    constexpr float kLog2e = 1.4426950408889634f;
+    bool ok = true;
+    for (int it = 0; it < niter; ++it) {
+      const uint32_t par = it & 1;
+      const int q0 = 128 * (i_begin + it);
+      // stage LSE (base 2) and D of this query tile; rows past the sequence get
+      // LSE = +inf so their P is exactly 0
+      {
+        const int q = q0 + t;
+        float lv = INFINITY, dv = 0.f;
+        if (q < L) {
+          const size_t li = VARLEN ? (static_cast<size_t>(h) * p.total + tok0 + q)
+                                   : ((static_cast<size_t>(b) * p.H + h) * p.N + q);
+          lv = p.lse[li] * kLog2e;
+          dv = p.dvec[li];
+        }
+        named_bar_sync(1, 128);  // everyone is done with the previous tile's values
+        sLSE[t] = lv;
+        sDv[t] = dv;
+        named_bar_sync(1, 128);
+      }
+      ok = mbar_wait(bar(C::BAR_S), par, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const bool diag = CAUSAL && (q0 == k0);
+      uint32_t pk[4][16];
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t s[32];
+        tmem_ld32(lane_base + C::TM_S + 32 * cc, s);
+        tmem_wait_ld(s);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int qa = 32 * cc + 2 * i;
+          float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -sLSE[qa]));
+          float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -sLSE[qa + 1]));
+          if (diag) {
+            if (t > qa) p0 = 0.f;
+            if (t > qa + 1) p1 = 0.f;
+          }
+          if (!key_ok) p0 = p1 = 0.f;
+          pk[cc][i] = pack_bf16x2(p0, p1);
+        }
+      }
+      // P^T (bf16) into the first 64 columns of the S^T block; every S^T value
+      // has been read above
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) tmem_st16(lane_base + C::TM_S + 16 * cc, pk[cc]);
+      tmem_wait_st();
+      tc_fence_before();
+      mbar_arrive(bar(C::BAR_P));
+      // dS^T = P^T (dP^T - D)
+      ok = mbar_wait(bar(C::BAR_DP), par, abort_flag) && mbar_wait(bar(C::BAR_DS_EMPTY), par ^ 1u, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) {
+        ok = false;
+        break;
+      }
+      tc_fence_after();
+      const uint32_t sDS = sbase + C::OFF_DS;
+#pragma unroll
+      for (int cc = 0; cc < 4; ++cc) {
+        uint32_t dp[32];
+        tmem_ld32(lane_base + C::TM_DP + 32 * cc, dp);
+        tmem_wait_ld(dp);
+        uint32_t w[16];
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          const int qa = 32 * cc + 2 * i;
+          const float d0 = bf16lo_to_f32(pk[cc][i]) * (__uint_as_float(dp[2 * i]) - sDv[qa]);
+          const float d1 = bf16hi_to_f32(pk[cc][i]) * (__uint_as_float(dp[2 * i + 1]) - sDv[qa + 1]);
+          w[i] = pack_bf16x2(d0, d1);
+        }
+        // queries 32cc..32cc+31 -> 64-query region cc/2, 16-byte chunks (cc&1)*4 + 0..3
+        const uint32_t region = sDS + (cc >> 1) * 16384;
+#pragma unroll
+        for (int u = 0; u < 4; ++u)
+          st_shared_v4(region + sw128_offset(t, (cc & 1) * 4 + u), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+      }
+      fence_proxy_async_smem();
+      tc_fence_before();
+      mbar_arrive(bar(C::BAR_DS));
+    }
+    // final dK, dV rows
+    if (ok) {
+      ok = mbar_wait(bar(C::BAR_ACC), 0, abort_flag);
+      if (__all_sync(0xffffffffu, ok)) {
+        tc_fence_after();
+        const size_t row = ((VARLEN ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.N) + key) * p.H + h;
+        __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(p.dk) + row * D;
+        __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(p.dv) + row * D;
+#pragma unroll 1
+        for (int which = 0; which < 2; ++which) {
+          const uint32_t col = which ? C::TM_DV : C::TM_DK;
+          const float mul = which ? 1.f : p.scale;
+          __nv_bfloat16* dst = which ? dvrow : dkrow;
+#pragma unroll 1
+          for (int cc = 0; cc < D / 32; ++cc) {
+            uint32_t a[32];
+            tmem_ld32(lane_base + col + 32 * cc, a);
+            tmem_wait_ld(a);
+            uint32_t w[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i)
+              w[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
+            if (key_ok) {
+#pragma unroll
+              for (int u = 0; u < 4; ++u) st_global_v4(dst + 32 * cc + 8 * u, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+            }
+          }
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------ dQ_i drain
+    const int t = threadIdx.x - 128;  // query row within the tile == tensor-memory lane
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+    for (int it = 0; it < niter; ++it) {
+      const uint32_t par = it & 1;
+      const int q = 128 * (i_begin + it) + t;
+      bool ok = mbar_wait(bar(C::BAR_DQ_FULL), par, abort_flag);
+      if (!__all_sync(0xffffffffu, ok)) break;
+      tc_fence_after();
+      float* dst = p.dq_acc + (((VARLEN ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.N) + q) * p.H + h) * D;
+#pragma unroll 1
+      for (int cc = 0; cc < D / 32; ++cc) {
+        uint32_t a[32];
+        tmem_ld32(lane_base + C::TM_DQ + 32 * cc, a);
+        tmem_wait_ld(a);
+        if (q < L) {
+#pragma unroll
+          for (int u = 0; u < 8; ++u)
+            atomicAdd(reinterpret_cast<float4*>(dst + 32 * cc + 4 * u),
+                      make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
+                                  __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3])));
+        }
+      }
+      tc_fence_before();
+      mbar_arrive(bar(C::BAR_DQ_EMPTY));
+    }
+  }
+
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 9) {
+    tc_fence_after();
+    tmem_dealloc(tmem, C::TMEM_COLS);
+  }
+}
+
+}  // namespace fa

@@ -1,0 +1,115 @@
+/*
+ * fa.h -- C ABI of the B200 (sm_100a) exact-attention library.
+ *
+ * What it computes.  Exact scaled-dot-product attention,
+ *     O = softmax(scale * Q K^T  [+ causal mask]) V,
+ * with the per-row logsumexp, and its gradients.  The computation is tiled
+ * through on-chip memory and never writes the N x N score matrix to HBM
+ * ("FlashAttention: Fast and Memory-Efficient Exact Attention with
+ * IO-Awareness", sections "Ideas clave: Tiling" and "Softmax en linea";
+ * "FlashAttention" (aiunderstanding.org), section "Apercu technique").  The
+ * backward pass recomputes the attention blocks from Q, K and the stored
+ * logsumexp instead of storing them (same AI Atlas page, "Recalcular en vez de
+ * guardar"; "FlashAttention" (freenetmedia.pl), section "Jak dzialaja
+ * FlashAttention?").  Packed variable-length batches follow "Flash Attention"
+ * (docs.monostate.ai), section "Con Sequence Packing": each packed sequence
+ * attends only to itself.
+ *
+ * Conventions (the pages give no equations; these are the plain readings):
+ *   - scale is a caller-supplied float, normally 1/sqrt(d);
+ *   - causal: query i sees key j iff j <= i, positions local to the sequence;
+ *   - LSE_i = ln sum_j exp(scale * q_i . k_j) over unmasked j (natural log);
+ *   - dense tensors Q, K, V, O, dO, dQ, dK, dV: contiguous bf16 [B, N, H, d]
+ *     (head dim innermost); dense LSE and the D vector: fp32 [B, H, N];
+ *   - packed tensors: contiguous bf16 [total, H, d]; packed LSE: fp32 [H, total];
+ *     cu_seqlens: int32 device array of nseq+1 non-decreasing prefix offsets
+ *     with cu_seqlens[0] = 0 and cu_seqlens[nseq] = total;
+ *   - head dim d is 64 or 128; bf16 inputs, fp32 accumulation and softmax.
+ *
+ * Ownership.  Every pointer is a DEVICE pointer owned by the caller, 16-byte
+ * aligned, on the current CUDA device.  The library never allocates device
+ * memory: the backward pass takes a caller-allocated workspace of
+ * fa_bwd_workspace_size() bytes.  Outputs are fully overwritten; the
+ * workspace holds no state between calls.  All calls are asynchronous on
+ * `stream` (a cudaStream_t; NULL = legacy default stream) and return after
+ * the launch; errors found on the host are returned before anything is
+ * launched.  Calls are thread-safe.
+ *
+ * Errors.  FA_ERR_INVALID_ARG for a null or misaligned pointer, a size < 1
+ * or too large, or a too-small workspace; FA_ERR_UNSUPPORTED for d not in
+ * {64, 128} or a device that is not compute capability 10.0 (sm_100); FA_ERR_CUDA
+ * when a CUDA call or launch fails.  Every on-device pipeline wait is bounded:
+ * an expired wait ends the kernel and sets a device error word, which
+ * fa_get_device_error() reports as FA_ERR_TIMEOUT.  The library never calls
+ * exit, abort or __trap.
+ */
+#ifndef FA_B200_H
+#define FA_B200_H
+
+#include <stddef.h>
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+typedef enum {
+  FA_OK = 0,
+  FA_ERR_INVALID_ARG = 1,
+  FA_ERR_UNSUPPORTED = 2,
+  FA_ERR_CUDA = 3,
+  FA_ERR_TIMEOUT = 4,
+  FA_ERR_WORKSPACE = 5
+} fa_status;
+
+/* Forward, dense batch.
+ * q, k, v: bf16 [B, N, H, d] inputs.  o: bf16 [B, N, H, d] output.
+ * lse: fp32 [B, H, N] output (natural-log logsumexp of each query row).
+ * causal: 0 or 1.  One fused kernel; no N x N buffer exists at any point. */
+fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                 int B, int N, int H, int d, float scale, int causal, void* stream);
+
+/* Forward, packed variable-length batch.
+ * q, k, v, o: bf16 [total, H, d]; lse: fp32 [H, total]; cu_seqlens: int32
+ * device array [nseq + 1]; max_seqlen >= every sequence length (used to size
+ * the launch; sequences longer than it are an error the kernel cannot see,
+ * so pass the true maximum). */
+fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse,
+                        const int* cu_seqlens, int nseq, int total, int max_seqlen,
+                        int H, int d, float scale, int causal, void* stream);
+
+/* Bytes of workspace the backward pass needs for rows = B*N (dense) or
+ * rows = total (packed): an fp32 dQ accumulator [rows, H, d] plus the fp32
+ * D = rowsum(dO * O) vector [rows * H], each 256-byte aligned.  Returns 0
+ * for invalid sizes. */
+size_t fa_bwd_workspace_size(int B, int N, int H, int d);
+
+/* Backward, dense batch.
+ * q, k, v, o, dO: bf16 [B, N, H, d] (o and lse exactly as fa_fwd returned them);
+ * lse: fp32 [B, H, N].  dq, dk, dv: bf16 [B, N, H, d] outputs.
+ * workspace: device buffer of ws_bytes >= fa_bwd_workspace_size(B, N, H, d).
+ * P is recomputed tile by tile from Q, K and lse; dQ is accumulated in fp32
+ * in the workspace and cast to bf16 at the end. */
+fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                 const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                 int B, int N, int H, int d, float scale, int causal, void* stream);
+
+/* Backward, packed variable-length batch.  Layouts as fa_varlen_fwd;
+ * ws_bytes >= fa_bwd_workspace_size(1, total, H, d). */
+fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                        const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                        const int* cu_seqlens, int nseq, int total, int max_seqlen,
+                        int H, int d, float scale, int causal, void* stream);
+
+/* Static text for a status code (never NULL). */
+const char* fa_status_string(fa_status s);
+
+/* Synchronises `stream`, then reads and clears this device's error word.
+ * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
+ * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK. */
+fa_status fa_get_device_error(void* stream);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* FA_B200_H */
