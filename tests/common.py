@@ -15,8 +15,18 @@ def f64(t: torch.Tensor) -> np.ndarray:
     return t.detach().float().cpu().numpy().astype(np.float64)
 
 
+GRAD_ATOL_WHEN_ZERO = 1e-3
+
+
 def rel_fro(a: np.ndarray, b: np.ndarray) -> float:
-    return float(np.linalg.norm(a - b) / max(np.linalg.norm(b), 1e-30))
+    """Relative Frobenius error.  Where the exact gradient is identically zero
+    (a single key: softmax of one entry has zero derivative) the ratio is
+    undefined; there the error is the max-abs deviation scaled so that the
+    same 5e-2 bar means max|a| <= 1e-3."""
+    nb = float(np.linalg.norm(b))
+    if nb == 0.0:
+        return float(np.max(np.abs(a))) * (5e-2 / GRAD_ATOL_WHEN_ZERO) if a.size else 0.0
+    return float(np.linalg.norm(a - b) / nb)
 
 
 def max_abs(a: np.ndarray, b: np.ndarray) -> float:
