@@ -1,0 +1,372 @@
+#!/usr/bin/env python3
+"""Throughput of the exact-attention hot path on B200: one step = forward +
+backward of the fused kernels over one batch of synthetic input.
+
+Workload (default): B=4, H=16, N=4096, d=128, causal, bf16 Q/K/V/dO i.i.d.
+N(0,1) with Q and K doubled (softmax range stress) -- the forward+backward
+workload at N >= 4096, d = 128 on which the performance target is stated.
+Metric: attention TFLOP/s of forward + backward, with the algorithmic FLOP
+count 4 B H N^2 d for the forward (halved for causal) and 2.5x that for the
+backward.
+
+Timing: W untimed warm-up steps, then K steps bracketed by a barrier and a
+device synchronize, timed with CUDA events on the launching stream; multi-GPU
+runs report the max over ranks.  The inputs (256 MiB of bf16) are larger than
+the 126 MB L2, so no flush is needed between steps.  SM clocks and throttle
+reasons are sampled with nvidia-smi during the timed region.
+
+Lines printed: one JSON object (rank 0).  `--impl reference` times the fp64
+CPU oracle instead (the slow baseline), on a bounded sample of the same
+workload.
+"""
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import math
+import os
+import re
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import torch  # noqa: E402
+
+from workloads import WORKLOADS, make_dense  # noqa: E402
+
+WORKLOAD = "fwd_bwd_causal_b4_h16_n4096_d128_qk2x"
+METRIC = "attention TFLOP/s fwd+bwd (bf16), fraction of B200 dense BF16 peak"
+UNIT = "TFLOP/s"
+
+
+def fwd_flops(B, N, H, d, causal):
+    f = 4.0 * B * H * N * N * d
+    return f / 2 if causal else f
+
+
+def load_peaks():
+    try:
+        with open(os.path.join(ROOT, "MEASURED_PEAKS.json")) as f:
+            p = json.load(f)
+        return {"bf16_tflops": float(p["bf16_tflops"]), "bf16_tflops_sustained": float(p["bf16_tflops_sustained"]),
+                "hbm_gbs": float(p["hbm_gbs"]), "source": "measured"}
+    except Exception:
+        return {"bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "hbm_gbs": 6650.0, "source": "fallback"}
+
+
+def kernel_source_sha() -> str:
+    h = hashlib.sha256()
+    for f in ("fa_bwd.cuh", "fa_fwd.cuh", "sm100_ptx.cuh", "fa_api.cu"):
+        with open(os.path.join(ROOT, "exact_io_aware_95_b200", "csrc", f), "rb") as fh:
+            h.update(fh.read())
+    return h.hexdigest()[:16]
+
+
+def recorded_traffic(kernel: str):
+    """DRAM bytes per launch from the committed ncu summary, if it was taken on
+    the current kernel sources (else None)."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.md")
+    if not os.path.exists(path):
+        return None
+    sha = kernel_source_sha()
+    for line in open(path):
+        m = re.match(r"\|\s*(\S+)\s*\|\s*(\S+)\s*\|\s*([0-9.eE+]+)\s*\|", line)
+        if m and m.group(1) == kernel and m.group(2) == sha:
+            return float(m.group(3))
+    return None
+
+
+class ClockSampler:
+    """nvidia-smi sampling of SM clock and throttle reasons during the timed region."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, device_index: int):
+        self.proc = None
+        self.tmp = None
+        self.dev = device_index
+
+    def start(self):
+        try:
+            self.tmp = tempfile.NamedTemporaryFile("w+", suffix=".csv", delete=False)
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.dev), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "50"], stdout=self.tmp, stderr=subprocess.DEVNULL)
+            time.sleep(0.5)  # let the sampler start producing before the timed region
+        except Exception:
+            self.proc = None
+
+    def stop(self):
+        if self.proc is None:
+            return None
+        self.proc.terminate()
+        try:
+            self.proc.wait(timeout=5)
+        except Exception:
+            self.proc.kill()
+        self.tmp.flush()
+        rows = []
+        with open(self.tmp.name) as f:
+            for line in f:
+                parts = [x.strip() for x in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.tmp.name)
+        if not rows:
+            return None
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        busy = [x for x in sm if x > 500] or sm
+        reasons = set()
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        for r in rows:
+            for n, v in zip(names, r[4:8]):
+                if v.lower() == "active":
+                    reasons.add(n)
+        return {"sm_mhz": statistics.median(busy) if busy else None,
+                "sm_max_mhz": float(rows[0][1]) if rows[0][1].replace(".", "").isdigit() else None,
+                "power_w_max": max(float(r[2]) for r in rows if r[2].replace(".", "").isdigit()),
+                "samples": len(rows), "reasons": sorted(reasons)}
+
+
+def cpu_cores() -> int:
+    try:
+        return len(os.sched_getaffinity(0))
+    except Exception:
+        return os.cpu_count() or 1
+
+
+_SAMPLE_CACHE = {}
+
+
+def oracle_sample(w, n_heads: int, seed: int = 0):
+    """Time the fp64 oracle (as it stands) on `n_heads` (b, h) heads of the
+    workload, forward + backward.  Returns (TFLOP/s, seconds, description)."""
+    import numpy as np
+    import oracle  # test infrastructure: only this baseline leg calls it
+
+    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)][:n_heads]
+    key = (w.name, n_heads, seed)
+    if key not in _SAMPLE_CACHE:
+        x = make_dense(w.B, w.N, w.H, w.d, seed=seed, qk_scale_factor=w.qk_scale_factor)
+        # the sampled heads only, as [1, N, n, d] float64 arrays
+        _SAMPLE_CACHE[key] = {k: np.stack([v[b, :, h].float().numpy() for b, h in heads], axis=1)[None]
+                              .astype(np.float64) for k, v in x.items()}
+    a = _SAMPLE_CACHE[key]
+    causal = True in w.causal
+    scale = 1.0 / math.sqrt(w.d)
+    t0 = time.perf_counter()
+    oracle.attn_fwd_ref(a["q"], a["k"], a["v"], scale, causal)
+    oracle.attn_bwd_ref(a["q"], a["k"], a["v"], a["do"], scale, causal)
+    dt = time.perf_counter() - t0
+    flops = 3.5 * fwd_flops(1, w.N, 1, w.d, causal) * len(heads)
+    return flops / dt / 1e12, dt, f"oracle fwd+bwd on {len(heads)} of {w.B * w.H} (b,h) heads, N={w.N}, d={w.d}"
+
+
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if torch.cuda.is_available() else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available():
+        torch.cuda.set_device(local)
+    return world, rank, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def allmax(x: float, world: int) -> float:
+    if world == 1:
+        return x
+    import torch.distributed as dist
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    t = torch.tensor([x], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+def run_reference(args, world, rank):
+    """The reference arm: the fp64 CPU oracle timed on the host cores."""
+    if rank != 0:
+        return None
+    w = WORKLOADS[WORKLOAD]
+    vals = []
+    for i in range(args.warmup + args.steps):
+        v, dt, desc = oracle_sample(w, 1)
+        if i >= args.warmup:
+            vals.append((v, dt))
+    value = statistics.mean(v for v, _ in vals)
+    ms = statistics.mean(dt for _, dt in vals) * 1e3
+    line = {"impl": "reference", "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": args.gpus,
+            "steps": args.steps, "warmup": args.warmup, "ms_per_step": ms, "higher_is_better": True,
+            "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
+            "config": {"workload": WORKLOAD, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "causal": True},
+            "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
+                             "sample": desc + " per step"},
+            "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
+    return line
+
+
+def run_gpu(args, world, rank, local):
+    import exact_io_aware_95_b200 as fa
+
+    w = WORKLOADS[WORKLOAD]
+    B, N, H, d = w.B, w.N, w.H, w.d
+    causal = True
+    scale = 1.0 / math.sqrt(d)
+    dev = torch.device("cuda", local)
+    host = make_dense(B, N, H, d, seed=args.seed + rank, qk_scale_factor=w.qk_scale_factor)
+    g = {k: v.to(dev) for k, v in host.items()}
+    o = torch.empty_like(g["q"])
+    lse = torch.empty((B, H, N), dtype=torch.float32, device=dev)
+    dq, dk, dv = torch.empty_like(g["q"]), torch.empty_like(g["k"]), torch.empty_like(g["v"])
+    ws = torch.empty(fa.workspace_size(B, N, H, d), dtype=torch.uint8, device=dev)
+    stream = torch.cuda.current_stream(dev)
+
+    def step():
+        fa.fwd(g["q"], g["k"], g["v"], causal=causal, scale=scale, out=o, lse=lse)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+
+    for _ in range(args.warmup):
+        step()
+    fa.check_device_error()
+    torch.cuda.synchronize(dev)
+
+    # ---- timed region: whole steps, plus per-call events for the per-kernel roofline
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    clocks = ClockSampler(local)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    t_start.record(stream)
+    for i in range(args.steps):
+        ev[i][0].record(stream)
+        fa.fwd(g["q"], g["k"], g["v"], causal=causal, scale=scale, out=o, lse=lse)
+        ev[i][1].record(stream)
+        fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv)
+        ev[i][2].record(stream)
+    t_end.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    clk = clocks.stop()
+    fa.check_device_error()
+    total_ms = allmax(t_start.elapsed_time(t_end), world)
+    fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
+    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    ms_step = total_ms / args.steps
+
+    ff = fwd_flops(B, N, H, d, causal)
+    bf = 2.5 * ff
+    value = (ff + bf) * world / (ms_step * 1e-3) / 1e12
+    fwd_tflops = ff / (fwd_ms * 1e-3) / 1e12
+    bwd_tflops = bf / (bwd_ms * 1e-3) / 1e12
+    peaks = load_peaks()
+
+    # ---- end to end through the public API with pinned host buffers
+    pin = {k: v.pin_memory() for k, v in host.items()}
+    out_h = {n: torch.empty(t.shape, dtype=t.dtype, pin_memory=True) for n, t in
+             (("o", o), ("lse", lse), ("dq", dq), ("dk", dk), ("dv", dv))}
+    h2d = sum(t.numel() * t.element_size() for t in pin.values())
+    d2h = sum(t.numel() * t.element_size() for t in out_h.values())
+
+    def e2e_step():
+        gg = {k: v.to(dev, non_blocking=True) for k, v in pin.items()}
+        oo, ll = fa.fwd(gg["q"], gg["k"], gg["v"], causal=causal, scale=scale)
+        a, b_, c = fa.bwd(gg["q"], gg["k"], gg["v"], oo, ll, gg["do"], causal=causal, scale=scale, workspace=ws)
+        for n, t in (("o", oo), ("lse", ll), ("dq", a), ("dk", b_), ("dv", c)):
+            out_h[n].copy_(t, non_blocking=True)
+
+    for _ in range(max(1, args.warmup)):
+        e2e_step()
+    torch.cuda.synchronize(dev)
+    e_steps = max(1, min(args.steps, 10))
+    s0, s1 = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+    barrier(world)
+    torch.cuda.synchronize(dev)
+    s0.record(stream)
+    for _ in range(e_steps):
+        e2e_step()
+    s1.record(stream)
+    torch.cuda.synchronize(dev)
+    barrier(world)
+    e2e_ms = allmax(s0.elapsed_time(s1), world) / e_steps
+    e2e_value = (ff + bf) * world / (e2e_ms * 1e-3) / 1e12
+
+    if rank != 0:
+        return None
+    line = {
+        "metric": METRIC, "value": value, "unit": UNIT, "n_gpus": world, "steps": args.steps,
+        "warmup": args.warmup, "ms_per_step": ms_step, "higher_is_better": True, "scaling": "weak",
+        "vs_baseline": None, "dtype": "bf16", "data": "synthetic",
+        "config": {"workload": WORKLOAD, "B": B, "N": N, "H": H, "d": d, "causal": causal,
+                   "qk_scale_factor": w.qk_scale_factor, "per_gpu_batch": B, "global_batch": B * world,
+                   "parallelism": f"replicas x{world} (independent (batch, head) shards)",
+                   "l2": "inputs (256 MiB bf16) larger than the 126 MB L2; no flush"},
+        "fwd_tflops": fwd_tflops, "bwd_tflops": bwd_tflops, "fwd_ms": fwd_ms, "bwd_ms": bwd_ms,
+        "frac_of_peak": {"step_vs_burst": value / world / peaks["bf16_tflops"],
+                         "fwd_vs_burst": fwd_tflops / peaks["bf16_tflops"],
+                         "bwd_vs_burst": bwd_tflops / peaks["bf16_tflops"],
+                         "peak_source": peaks["source"]},
+        "roofline": {"kernel": "fa_bwd call (preprocess + main + dq_convert launches)", "bound": "tensor",
+                     "achieved": bwd_tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                     "frac": bwd_tflops / peaks["bf16_tflops_sustained"],
+                     "peak_kind": f"sustained bf16 GEMM ({peaks['source']})",
+                     "traffic": recorded_traffic("fa_bwd_kernel")},
+        "roofline_fwd": {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_tflops,
+                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
+                         "frac": fwd_tflops / peaks["bf16_tflops_sustained"],
+                         "traffic": recorded_traffic("fa_fwd_kernel")},
+        "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
+                "ms_per_step": e2e_ms},
+        "gpu_launches": 4 * args.steps,
+        "clocks": clk,
+    }
+    if not args.no_cpu_baseline and world == 1:
+        v, dt, desc = oracle_sample(w, 2)
+        line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc,
+                                "seconds": dt}
+    return line
+
+
+def main():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=300)
+    ap.add_argument("--warmup", type=int, default=10)
+    ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    args = ap.parse_args()
+    if args.warmup < 3:
+        args.warmup = 3
+    world, rank, local = dist_setup(args)
+    try:
+        line = run_reference(args, world, rank) if args.impl == "reference" else run_gpu(args, world, rank, local)
+        if line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()

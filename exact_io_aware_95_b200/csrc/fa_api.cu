@@ -69,11 +69,23 @@ fa_status current_device(int* dev) {
   return st.checked == 1 ? FA_OK : FA_ERR_UNSUPPORTED;
 }
 
-// Set the dynamic shared-memory limit of `kern` once per device.
+// Set the dynamic shared-memory limit of `kern` once per device.  Kernels
+// that re-balance registers between warpgroups (setmaxnreg) must have been
+// compiled to exactly fa::kLaunchRegs registers per thread: their split adds
+// up to 384 * kLaunchRegs, and a split larger than the launch allocation
+// would never be granted.  Refuse to launch such a kernel otherwise.
 template <typename K>
-fa_status ensure_smem(K kern, int dev, int bytes, bool* done_flags) {
+fa_status ensure_smem(K kern, int dev, int bytes, bool* done_flags, int need_regs = 0) {
   std::lock_guard<std::mutex> lk(g_mu);
   if (!done_flags[dev]) {
+    if (need_regs) {
+      cudaFuncAttributes attr;
+      if (cudaFuncGetAttributes(&attr, kern) != cudaSuccess) {
+        cudaGetLastError();
+        return FA_ERR_CUDA;
+      }
+      if (attr.numRegs != need_regs) return FA_ERR_UNSUPPORTED;
+    }
     if (cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, bytes) != cudaSuccess) {
       cudaGetLastError();
       return FA_ERR_CUDA;
@@ -116,7 +128,7 @@ fa_status launch_fwd(int dev, const CUtensorMap& q, const CUtensorMap& k, const 
   constexpr bool PTM = FA_FWD_P_IN_TMEM;
   auto kern = fa::fa_fwd_kernel<D, CAUSAL, VARLEN, PTM>;
   constexpr int smem = fa::FwdCfg<D, PTM>::SMEM_BYTES;
-  fa_status st = ensure_smem(kern, dev, smem, done);
+  fa_status st = ensure_smem(kern, dev, smem, done, fa::kLaunchRegs);
   if (st != FA_OK) return st;
   const int64_t grid = static_cast<int64_t>(p.npairs) * p.B * p.H;
   if (grid <= 0 || grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
@@ -179,7 +191,7 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   static bool done[kMaxDevices] = {};
   auto kern = fa::fa_bwd_kernel<D, CAUSAL, VARLEN>;
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
-  fa_status st = ensure_smem(kern, dev, smem, done);
+  fa_status st = ensure_smem(kern, dev, smem, done, fa::kLaunchRegs);
   if (st != FA_OK) return st;
   // 1) D = rowsum(dO * O) and zeroed dQ accumulator
   {
@@ -201,7 +213,7 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
     const int64_t n8 = static_cast<int64_t>(p.rows) * p.H * D / 8;
     const int64_t blocks = (n8 + 255) / 256;
     if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
-    fa::fa_bwd_dq_convert_kernel<<<static_cast<unsigned>(blocks), 256, 0, s>>>(p.dq_acc, p.dq, n8, p.scale);
+    fa::fa_bwd_dq_convert_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
     if ((st = launch_status()) != FA_OK) return st;
   }
   return FA_OK;

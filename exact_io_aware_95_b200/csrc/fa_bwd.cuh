@@ -29,11 +29,14 @@
 // products.  The dQ product reads the same dS^T buffer through an MN-major
 // descriptor, so dS is written once.
 //
-// Warp roles of the main kernel (320 threads):
+// Warp roles of the main kernel (384 threads, three warpgroups):
 //   warps 0-3  P^T and dS^T (thread t = key row t), final dK/dV stores
 //   warps 4-7  dQ_i drain: tensor memory -> fp32 atomics (thread t = query row t)
 //   warp  8    TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring
 //   warp  9    tensor-memory allocator and the single MMA-issuing thread
+//   warps 10-11 idle
+// Registers: the producer/MMA warpgroup drops to 96, the P/dS warpgroup rises
+// to 224, the drain warpgroup keeps the launch value.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -46,7 +49,7 @@ struct BwdParams {
   void* dq;
   void* dk;
   void* dv;
-  float* dq_acc;  // fp32, same [rows, H, d] layout as dq
+  float* dq_acc;  // fp32 accumulator, column-block-major: see dq_acc_index()
   float* dvec;    // fp32 D, same indexing as lse
   const int* cu_seqlens;
   int B;         // dense: batch; packed: number of sequences
@@ -59,11 +62,25 @@ struct BwdParams {
   float scale_log2;
 };
 
+// The fp32 dQ accumulator is laid out so that 32 consecutive query rows of one
+// (batch entry, head) and one 4-column group are 512 contiguous bytes: float4
+// element ((bh * D/4 + g) * R + r), with bh = b*H + h and r = n, R = N for
+// dense batches, and bh = h, r = token, R = total for packed ones.  The dQ
+// drain (one thread per query row) then issues vector atomics that cover whole
+// 128-byte lines per warp instead of 32 scattered 16-byte pieces.
+__device__ __forceinline__ size_t dq_acc_index4(int bh, int g, int64_t r, int64_t R, int D) {
+  return (static_cast<size_t>(bh) * (D / 4) + g) * static_cast<size_t>(R) + static_cast<size_t>(r);
+}
+
 // ------------------------------------------------------------------ preprocess
-// One warp per (token, head) row.
+// One warp per (token, head) row computes D; every thread also zeroes one
+// float4 of the accumulator (linear order, layout independent).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams p) {
-  const int64_t w = (static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x) >> 5;
+  const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  const int64_t nacc4 = static_cast<int64_t>(p.rows) * p.H * (D / 4);
+  if (gtid < nacc4) reinterpret_cast<float4*>(p.dq_acc)[gtid] = make_float4(0.f, 0.f, 0.f, 0.f);
+  const int64_t w = gtid >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t nrows = static_cast<int64_t>(p.rows) * p.H;
   if (w >= nrows) return;
@@ -86,9 +103,6 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams 
   }
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  float* acc_row = p.dq_acc + base + lane * PER;
-#pragma unroll
-  for (int i = 0; i < PER; ++i) acc_row[i] = 0.f;
   if (lane == 0) {
     size_t li;
     if (p.cu_seqlens) {
@@ -102,18 +116,37 @@ __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams 
 }
 
 // ------------------------------------------------------------------ dQ convert
-__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const float* __restrict__ acc, void* dq, int64_t n8,
-                                                                 float scale) {
+// Thread i handles 8 columns (float4 groups 2k, 2k+1) of one (bh, row):
+// i = (bh * D/8 + k) * R + r, so a warp reads 32 consecutive rows of a group.
+template <int D>
+__global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams p) {
   const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  if (i >= n8) return;
-  const float4 a = reinterpret_cast<const float4*>(acc)[2 * i];
-  const float4 b = reinterpret_cast<const float4*>(acc)[2 * i + 1];
-  uint4 r;
-  r.x = pack_bf16x2(a.x * scale, a.y * scale);
-  r.y = pack_bf16x2(a.z * scale, a.w * scale);
-  r.z = pack_bf16x2(b.x * scale, b.y * scale);
-  r.w = pack_bf16x2(b.z * scale, b.w * scale);
-  reinterpret_cast<uint4*>(dq)[i] = r;
+  const int64_t R = p.cu_seqlens ? p.total : p.N;
+  const int64_t nbh = p.cu_seqlens ? p.H : static_cast<int64_t>(p.B) * p.H;
+  if (i >= nbh * (D / 8) * R) return;
+  const int64_t r = i % R;
+  const int64_t t = i / R;
+  const int k = static_cast<int>(t % (D / 8));
+  const int bh = static_cast<int>(t / (D / 8));
+  const float4* acc = reinterpret_cast<const float4*>(p.dq_acc);
+  const float4 a = acc[dq_acc_index4(bh, 2 * k, r, R, D)];
+  const float4 c = acc[dq_acc_index4(bh, 2 * k + 1, r, R, D)];
+  int64_t tok;
+  int h;
+  if (p.cu_seqlens) {
+    h = bh;
+    tok = r;
+  } else {
+    h = bh % p.H;
+    tok = static_cast<int64_t>(bh / p.H) * p.N + r;
+  }
+  const float sc = p.scale;
+  uint4 o;
+  o.x = pack_bf16x2(a.x * sc, a.y * sc);
+  o.y = pack_bf16x2(a.z * sc, a.w * sc);
+  o.z = pack_bf16x2(c.x * sc, c.y * sc);
+  o.w = pack_bf16x2(c.z * sc, c.w * sc);
+  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(tok) * p.H + h) * D + 8 * k) = o;
 }
 
 // ------------------------------------------------------------------ main kernel
@@ -151,12 +184,12 @@ struct BwdCfg {
   static constexpr bool DQ_ALIASES_DP = (256 + 2 * D + D) > 512;
   static constexpr int TM_DQ = DQ_ALIASES_DP ? TM_DP : 256 + 2 * D;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int D, bool CAUSAL, bool VARLEN>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const BwdParams p) {
@@ -224,7 +257,9 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    regs_dec<96>();
+  }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -267,17 +302,8 @@ __global__ void __launch_bounds__(320, 1)
       constexpr uint32_t kIdSq = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdDV = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK
       constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, true, true);      // dQ: A = dS (MN-major view)
-      bool ok = mbar_wait(bar(C::BAR_KV), 0, abort_flag);
-      if (ok) tc_fence_after();
-      for (int it = 0; ok && it < niter; ++it) {
-        const int st = it % C::NSTAGE;
-        const uint32_t ph = (it / C::NSTAGE) & 1;
-        const uint32_t par = it & 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
-        const uint32_t sdO = sbase + C::OFF_DO + st * C::TILE_BYTES;
-        if (!(ok = mbar_wait(bar(C::BAR_QDO_FULL + st), ph, abort_flag))) break;
-        tc_fence_after();
-        // S^T = K Q^T
+      auto issue_s = [&](int it) {  // S^T = K Q_it^T
+        const uint32_t sQ = sbase + C::OFF_Q + (it % C::NSTAGE) * C::TILE_BYTES;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
@@ -285,7 +311,28 @@ __global__ void __launch_bounds__(320, 1)
                   kIdSq, kk > 0);
         }
         umma_commit(bar(C::BAR_S));
-        // dP^T = V dO^T  (its columns may hold the previous dQ_i: wait until drained)
+      };
+      // Order per query tile i:  dV(i)  dP^T(i)  S^T(i+1)  dK(i)  dQ(i)
+      // so that P^T(i+1) is computed while dK(i) and dQ(i) run, and dS^T(i)
+      // while S^T(i+1) runs.
+      bool ok = mbar_wait(bar(C::BAR_KV), 0, abort_flag) && mbar_wait(bar(C::BAR_QDO_FULL), 0, abort_flag);
+      if (ok) {
+        tc_fence_after();
+        issue_s(0);
+      }
+      for (int it = 0; ok && it < niter; ++it) {
+        const int st = it % C::NSTAGE;
+        const uint32_t par = it & 1;
+        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
+        const uint32_t sdO = sbase + C::OFF_DO + st * C::TILE_BYTES;
+        // dV += P^T dO   (A = P^T packed bf16 in tensor memory)
+        if (!(ok = mbar_wait(bar(C::BAR_P), par, abort_flag))) break;
+        tc_fence_after();
+#pragma unroll
+        for (int kk = 0; kk < 8; ++kk)
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdDV,
+                  (it > 0 || kk > 0));
+        // dP^T = V dO^T  (its columns may hold the previous dQ tile: wait until drained)
         if (C::DQ_ALIASES_DP && it > 0) {
           if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
           tc_fence_after();
@@ -297,13 +344,13 @@ __global__ void __launch_bounds__(320, 1)
                   kIdSq, kk > 0);
         }
         umma_commit(bar(C::BAR_DP));
-        // dV += P^T dO   (A = P^T packed bf16 in tensor memory)
-        if (!(ok = mbar_wait(bar(C::BAR_P), par, abort_flag))) break;
-        tc_fence_after();
-#pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdDV,
-                  (it > 0 || kk > 0));
+        // S^T of the next query tile (P^T(i) was consumed by dV above, in issue order)
+        if (it + 1 < niter) {
+          const int st1 = (it + 1) % C::NSTAGE;
+          if (!(ok = mbar_wait(bar(C::BAR_QDO_FULL + st1), ((it + 1) / C::NSTAGE) & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_s(it + 1);
+        }
         // dK += dS^T Q ;  dQ_i = dS K
         if (!(ok = mbar_wait(bar(C::BAR_DS), par, abort_flag))) break;
         tc_fence_after();
@@ -333,6 +380,7 @@ __global__ void __launch_bounds__(320, 1)
     __syncwarp();
   } else if (warp < 4) {
     // ------------------------------------------------------------ P^T and dS^T
+    regs_inc<224>();
     const int t = threadIdx.x;  // key row within the tile == tensor-memory lane
     const int key = k0 + t;
     const bool key_ok = key < L;
@@ -342,25 +390,29 @@ __global__ void __launch_bounds__(320, 1)
     const float c = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     bool ok = true;
+    // LSE (base 2) and D of query row q of the tile starting at q0; rows past
+    // the sequence get LSE = +inf so their P is exactly 0.
+    auto fetch = [&](int q0, float& lv, float& dv) {
+      const int q = q0 + t;
+      lv = INFINITY;
+      dv = 0.f;
+      if (q < L) {
+        const size_t li = VARLEN ? (static_cast<size_t>(h) * p.total + tok0 + q)
+                                 : ((static_cast<size_t>(b) * p.H + h) * p.N + q);
+        lv = p.lse[li] * kLog2e;
+        dv = p.dvec[li];
+      }
+    };
+    float lv_next, dv_next;
+    fetch(128 * i_begin, lv_next, dv_next);
     for (int it = 0; it < niter; ++it) {
       const uint32_t par = it & 1;
       const int q0 = 128 * (i_begin + it);
-      // stage LSE (base 2) and D of this query tile; rows past the sequence get
-      // LSE = +inf so their P is exactly 0
-      {
-        const int q = q0 + t;
-        float lv = INFINITY, dv = 0.f;
-        if (q < L) {
-          const size_t li = VARLEN ? (static_cast<size_t>(h) * p.total + tok0 + q)
-                                   : ((static_cast<size_t>(b) * p.H + h) * p.N + q);
-          lv = p.lse[li] * kLog2e;
-          dv = p.dvec[li];
-        }
-        named_bar_sync(1, 128);  // everyone is done with the previous tile's values
-        sLSE[t] = lv;
-        sDv[t] = dv;
-        named_bar_sync(1, 128);
-      }
+      named_bar_sync(1, 128);  // everyone is done with the previous tile's values
+      sLSE[t] = lv_next;
+      sDv[t] = dv_next;
+      named_bar_sync(1, 128);
+      if (it + 1 < niter) fetch(q0 + 128, lv_next, dv_next);  // lands during this tile
       ok = mbar_wait(bar(C::BAR_S), par, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
         ok = false;
@@ -368,6 +420,7 @@ __global__ void __launch_bounds__(320, 1)
       }
       tc_fence_after();
       const bool diag = CAUSAL && (q0 == k0);
+      const float4* sLSE4 = reinterpret_cast<const float4*>(sLSE);
       uint32_t pk[4][16];
 #pragma unroll
       for (int cc = 0; cc < 4; ++cc) {
@@ -375,16 +428,22 @@ __global__ void __launch_bounds__(320, 1)
         tmem_ld32(lane_base + C::TM_S + 32 * cc, s);
         tmem_wait_ld(s);
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int qa = 32 * cc + 2 * i;
-          float p0 = ex2(fmaf(__uint_as_float(s[2 * i]), c, -sLSE[qa]));
-          float p1 = ex2(fmaf(__uint_as_float(s[2 * i + 1]), c, -sLSE[qa + 1]));
+        for (int m = 0; m < 8; ++m) {
+          const float4 l4 = sLSE4[8 * cc + m];
+          const int qa = 32 * cc + 4 * m;
+          float p0 = ex2(fmaf(__uint_as_float(s[4 * m + 0]), c, -l4.x));
+          float p1 = ex2(fmaf(__uint_as_float(s[4 * m + 1]), c, -l4.y));
+          float p2 = ex2(fmaf(__uint_as_float(s[4 * m + 2]), c, -l4.z));
+          float p3 = ex2(fmaf(__uint_as_float(s[4 * m + 3]), c, -l4.w));
           if (diag) {
             if (t > qa) p0 = 0.f;
             if (t > qa + 1) p1 = 0.f;
+            if (t > qa + 2) p2 = 0.f;
+            if (t > qa + 3) p3 = 0.f;
           }
-          if (!key_ok) p0 = p1 = 0.f;
-          pk[cc][i] = pack_bf16x2(p0, p1);
+          if (!key_ok) p0 = p1 = p2 = p3 = 0.f;
+          pk[cc][2 * m] = pack_bf16x2(p0, p1);
+          pk[cc][2 * m + 1] = pack_bf16x2(p2, p3);
         }
       }
       // P^T (bf16) into the first 64 columns of the S^T block; every S^T value
@@ -407,13 +466,18 @@ __global__ void __launch_bounds__(320, 1)
         uint32_t dp[32];
         tmem_ld32(lane_base + C::TM_DP + 32 * cc, dp);
         tmem_wait_ld(dp);
+        const float4* sDv4 = reinterpret_cast<const float4*>(sDv);
         uint32_t w[16];
 #pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const int qa = 32 * cc + 2 * i;
-          const float d0 = bf16lo_to_f32(pk[cc][i]) * (__uint_as_float(dp[2 * i]) - sDv[qa]);
-          const float d1 = bf16hi_to_f32(pk[cc][i]) * (__uint_as_float(dp[2 * i + 1]) - sDv[qa + 1]);
-          w[i] = pack_bf16x2(d0, d1);
+        for (int m = 0; m < 8; ++m) {
+          const float4 d4 = sDv4[8 * cc + m];
+          const uint32_t a0 = pk[cc][2 * m], a1 = pk[cc][2 * m + 1];
+          const float d0 = bf16lo_to_f32(a0) * (__uint_as_float(dp[4 * m + 0]) - d4.x);
+          const float d1 = bf16hi_to_f32(a0) * (__uint_as_float(dp[4 * m + 1]) - d4.y);
+          const float d2 = bf16lo_to_f32(a1) * (__uint_as_float(dp[4 * m + 2]) - d4.z);
+          const float d3 = bf16hi_to_f32(a1) * (__uint_as_float(dp[4 * m + 3]) - d4.w);
+          w[2 * m] = pack_bf16x2(d0, d1);
+          w[2 * m + 1] = pack_bf16x2(d2, d3);
         }
         // queries 32cc..32cc+31 -> 64-query region cc/2, 16-byte chunks (cc&1)*4 + 0..3
         const uint32_t region = sDS + (cc >> 1) * 16384;
@@ -455,7 +519,7 @@ __global__ void __launch_bounds__(320, 1)
         }
       }
     }
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ dQ_i drain
     const int t = threadIdx.x - 128;  // query row within the tile == tensor-memory lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -465,7 +529,11 @@ __global__ void __launch_bounds__(320, 1)
       bool ok = mbar_wait(bar(C::BAR_DQ_FULL), par, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
-      float* dst = p.dq_acc + (((VARLEN ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.N) + q) * p.H + h) * D;
+      // accumulator rows: (bh, float4 group g, r) with r consecutive across the warp
+      const int bh = VARLEN ? h : b * p.H + h;
+      const int64_t R = VARLEN ? p.total : p.N;
+      const int64_t r = static_cast<int64_t>(VARLEN ? tok0 : 0) + q;
+      float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
 #pragma unroll 1
       for (int cc = 0; cc < D / 32; ++cc) {
         uint32_t a[32];
@@ -474,7 +542,7 @@ __global__ void __launch_bounds__(320, 1)
         if (q < L) {
 #pragma unroll
           for (int u = 0; u < 8; ++u)
-            atomicAdd(reinterpret_cast<float4*>(dst + 32 * cc + 4 * u),
+            atomicAdd(acc4 + dq_acc_index4(bh, 8 * cc + u, r, R, D),
                       make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
                                   __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3])));
         }

@@ -14,12 +14,15 @@
 // matrix is never formed ("FlashAttention: Fast and Memory-Efficient Exact
 // Attention with IO-Awareness", sections "Tiling" and "Softmax en linea").
 //
-// Warp roles (320 threads):
+// Warp roles (384 threads, three warpgroups):
 //   warps 0-3  softmax for query tile 0 (thread t owns row t: the tcgen05
 //              32x32b tensor-memory layout gives each thread one row)
 //   warps 4-7  softmax for query tile 1
 //   warp  8    TMA producer: Q0, Q1 once, then K_j, V_j into an NSTAGE ring
 //   warp  9    tensor-memory allocator and the single MMA-issuing thread
+//   warps 10-11 idle
+// The producer/MMA warpgroup gives up registers (56 each) so the two softmax
+// warpgroups can hold a whole 128-column score row (224 each).
 // The split of the non-matmul work into its own warps, so the MMA unit never
 // waits on it more than necessary, is the B200 form of "FlashAttention-2
 // (PT)", sections "1. Minimizacao de operacoes nao matriciais" and "3. Divisao
@@ -78,7 +81,7 @@ struct FwdCfg {
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
   static constexpr int TMEM_COLS = 512;                    // S0 | S1 | O0 | O1
   static constexpr int TM_S = 0, TM_O = 256;
-  static constexpr int THREADS = 320;
+  static constexpr int THREADS = 384;
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -86,7 +89,7 @@ constexpr float kRescaleThreshold = 8.0f;  // log2 units
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D, bool CAUSAL, bool VARLEN, bool PTM>
-__global__ void __launch_bounds__(320, 1)
+__global__ void __launch_bounds__(384, 1)
     fa_fwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const FwdParams p) {
   using C = FwdCfg<D, PTM>;
@@ -154,7 +157,9 @@ __global__ void __launch_bounds__(320, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-
+  if (warp >= 8) {
+    regs_dec<56>();
+  }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
@@ -279,8 +284,9 @@ __global__ void __launch_bounds__(320, 1)
       }
     }
     __syncwarp();
-  } else {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
+    regs_inc<224>();
     const int k = warp >> 2;
     const int t = threadIdx.x & 127;  // row within the query tile == tensor-memory lane
     const int nk = ntile[k];

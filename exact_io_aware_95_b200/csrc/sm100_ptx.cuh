@@ -262,3 +262,19 @@ __device__ __forceinline__ void named_bar_sync(int id, int count) {
 __device__ __forceinline__ float bf16lo_to_f32(uint32_t w) { return __uint_as_float(w << 16); }
 __device__ __forceinline__ float bf16hi_to_f32(uint32_t w) { return __uint_as_float(w & 0xffff0000u); }
 }  // namespace fa
+
+namespace fa {
+// Per-warpgroup register re-allocation (all four warps of a warpgroup execute
+// the same instruction).  The kernels that use it launch 384 threads with
+// exactly kLaunchRegs registers each (checked on the host before launch), so
+// the register file they draw on is 384 * kLaunchRegs = 64512.
+constexpr int kLaunchRegs = 168;
+template <int N>
+__device__ __forceinline__ void regs_inc() {
+  asm volatile("setmaxnreg.inc.sync.aligned.u32 %0;" ::"n"(N));
+}
+template <int N>
+__device__ __forceinline__ void regs_dec() {
+  asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
+}
+}  // namespace fa
