@@ -120,6 +120,16 @@ fa_status launch_status() {
 
 constexpr float kLog2e = 1.4426950408889634f;
 
+// Heads per scheduling group: as many as keep `bytes_per_head` of streamed
+// operands within a share of the 126 MB L2, at least 1, at most all heads.
+int head_group(int64_t bytes_per_head, int64_t heads) {
+  constexpr int64_t kL2Budget = 48ll << 20;
+  int64_t g = bytes_per_head > 0 ? kL2Budget / bytes_per_head : heads;
+  if (g < 1) g = 1;
+  if (g > heads) g = heads;
+  return static_cast<int>(g);
+}
+
 // ------------------------------------------------------------------ forward
 template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch_fwd(int dev, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
@@ -172,6 +182,7 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
   p.H = H;
   p.total = varlen ? total : N;
   p.npairs = (N + 255) / 256;
+  p.group = head_group(static_cast<int64_t>(N) * d * 2 * 2, static_cast<int64_t>(B) * H);  // K and V of one head
   p.scale_log2 = scale * kLog2e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   return d == 64 ? dispatch_fwd<64>(dev, causal, varlen, mq, mk, mv, p, s)
@@ -269,6 +280,7 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.total = varlen ? total : N;
   p.rows = static_cast<int>(rows * outer);
   p.nkvtiles = (N + 127) / 128;
+  p.group = head_group(static_cast<int64_t>(N) * d * (2 + 2 + 4), static_cast<int64_t>(B) * H);  // Q, dO, dQ acc
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

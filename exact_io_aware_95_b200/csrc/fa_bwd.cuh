@@ -58,6 +58,7 @@ struct BwdParams {
   int total;     // packed: total tokens; dense: N
   int rows;      // B*N (dense) or total (packed)
   int nkvtiles;  // ceil(N / 128)
+  int group;     // heads per scheduling group (L2-sized), >= 1
   float scale;
   float scale_log2;
 };
@@ -200,13 +201,18 @@ __global__ void __launch_bounds__(384, 1)
   const int warp = threadIdx.x >> 5;
   const int lane = threadIdx.x & 31;
 
-  // ---- work item: (key tile j, batch entry or sequence, head); longest key tiles first
-  int x = blockIdx.x;
-  const int h = x % p.H;
-  x /= p.H;
-  const int b = x % p.B;
-  x /= p.B;
-  const int j = x;
+  // ---- work item: (key tile j, batch entry or sequence, head).  Heads are taken
+  // in groups of p.group, sized on the host so that a group's Q, dO and dQ
+  // accumulator rows stay in L2; inside a group the key tiles go longest-first
+  // (causal) across all of its heads.
+  const int nbh = p.B * p.H;
+  const int g = blockIdx.x / (p.group * p.nkvtiles);
+  const int gs = min(p.group, nbh - g * p.group);
+  const int cidx = blockIdx.x - g * p.group * p.nkvtiles;
+  const int bh = g * p.group + cidx % gs;
+  const int j = cidx / gs;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
   int L, tok0, bcoord;
   if (VARLEN) {
     tok0 = p.cu_seqlens[b];

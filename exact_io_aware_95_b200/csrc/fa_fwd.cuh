@@ -50,6 +50,7 @@ struct FwdParams {
   int H;
   int total;              // packed: total tokens (row stride of LSE); dense: N
   int npairs;             // ceil(N / 256): 256-row query blocks per (sequence, head)
+  int group;              // heads per scheduling group (L2-sized), >= 1
   float scale_log2;       // scale * log2(e)
 };
 
@@ -69,13 +70,13 @@ struct FwdCfg {
   static constexpr int OFF_KV = OFF_Q + 2 * TILE_BYTES;
   static constexpr int OFF_P = OFF_KV + NSTAGE * TILE_BYTES;
   static constexpr int OFF_BAR = OFF_P + 2 * P_BYTES;
-  // barriers: q_full, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], p_full[2], drain
+  // barriers: q_full, kv_full[NSTAGE], kv_empty[NSTAGE], s_full[2], p_full[2][2 halves], drain
   static constexpr int BAR_Q = 0;
   static constexpr int BAR_KV_FULL = 1;
   static constexpr int BAR_KV_EMPTY = 1 + NSTAGE;
   static constexpr int BAR_S = 1 + 2 * NSTAGE;
   static constexpr int BAR_P = BAR_S + 2;
-  static constexpr int BAR_DRAIN = BAR_P + 2;
+  static constexpr int BAR_DRAIN = BAR_P + 4;
   static constexpr int NBAR = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;  // + alignment slack
@@ -100,12 +101,17 @@ __global__ void __launch_bounds__(384, 1)
   const int lane = threadIdx.x & 31;
 
   // ---- work item: (query block, batch entry or sequence, head); heavy blocks first
-  int x = blockIdx.x;
-  const int h = x % p.H;
-  x /= p.H;
-  const int b = x % p.B;
-  x /= p.B;
-  const int pair = p.npairs - 1 - x;
+  // Heads (batch entry or sequence, head) are taken in groups of p.group, sized
+  // on the host so that a group's K/V fit in L2; inside a group the query
+  // blocks go longest-first (causal) across all of its heads.
+  const int nbh = p.B * p.H;
+  const int g = blockIdx.x / (p.group * p.npairs);
+  const int gs = min(p.group, nbh - g * p.group);
+  const int c = blockIdx.x - g * p.group * p.npairs;
+  const int bh = g * p.group + c % gs;
+  const int pair = p.npairs - 1 - c / gs;
+  const int h = bh % p.H;
+  const int b = bh / p.H;
   int L, tok0, bcoord;
   if (VARLEN) {
     tok0 = p.cu_seqlens[b];
@@ -143,7 +149,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     for (int k = 0; k < 2; ++k) {
       mbar_init(bar(C::BAR_S + k), 1);
-      mbar_init(bar(C::BAR_P + k), 128);
+      mbar_init(bar(C::BAR_P + 2 * k), 128);
+      mbar_init(bar(C::BAR_P + 2 * k + 1), 128);
     }
     mbar_init(bar(C::BAR_DRAIN), 1);
     *abort_flag = 0;
@@ -211,9 +218,9 @@ __global__ void __launch_bounds__(384, 1)
           umma_ss(tmem + C::TM_S + 128 * k, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), kIdS, kk > 0);
         }
       };
-      auto issue_pv = [&](int k, int st, int j) {
+      auto issue_pv = [&](int k, int st, int j, int kk0) {
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk) {
+        for (int kk = kk0; kk < kk0 + 4; ++kk) {
           const uint32_t bb = sbase + C::OFF_KV + st * C::TILE_BYTES + kk * 2048;
           if constexpr (PTM) {
             umma_ts(tmem + C::TM_O + D * k, tmem + C::TM_S + 128 * k + kk * 8, sdesc_sw128(bb, 16384, 1024), kIdO,
@@ -258,9 +265,14 @@ __global__ void __launch_bounds__(384, 1)
         bool kready = false;
         for (int k = 0; ok && k < 2; ++k) {
           if (j >= ntile[k]) continue;
-          if (!(ok = mbar_wait(bar(C::BAR_P + k), j & 1, abort_flag))) break;
+          // P arrives in two halves of 64 keys; the first half's MMAs start
+          // while the softmax warps finish the second
+          if (!(ok = mbar_wait(bar(C::BAR_P + 2 * k), j & 1, abort_flag))) break;
           tc_fence_after();
-          issue_pv(k, vst, j);
+          issue_pv(k, vst, j, 0);
+          if (!(ok = mbar_wait(bar(C::BAR_P + 2 * k + 1), j & 1, abort_flag))) break;
+          tc_fence_after();
+          issue_pv(k, vst, j, 4);
           if (j + 1 < ntile[k]) {
             if (!kready) {
               if (!(ok = mbar_wait(bar(C::BAR_KV_FULL + nst), nph, abort_flag))) break;
@@ -321,15 +333,16 @@ __global__ void __launch_bounds__(384, 1)
             for (int i = 0; i < 32; ++i)
               if (kbase + 32 * cc + i > limit) s[cc][i] = __float_as_uint(-INFINITY);
         }
-        float mx0 = -INFINITY, mx1 = -INFINITY;
+        // row max: four independent chains of three-input maxima
+        float mx[4] = {-INFINITY, -INFINITY, -INFINITY, -INFINITY};
 #pragma unroll
         for (int cc = 0; cc < 4; ++cc)
 #pragma unroll
-          for (int i = 0; i < 32; i += 2) {
-            mx0 = fmaxf(mx0, __uint_as_float(s[cc][i]));
-            mx1 = fmaxf(mx1, __uint_as_float(s[cc][i + 1]));
-          }
-        const float mt = fmaxf(mx0, mx1) * c;
+          for (int i = 0; i < 32; i += 8)
+#pragma unroll
+            for (int a = 0; a < 4; ++a)
+              mx[a] = fmax3(mx[a], __uint_as_float(s[cc][i + 2 * a]), __uint_as_float(s[cc][i + 2 * a + 1]));
+        const float mt = fmaxf(fmaxf(mx[0], mx[1]), fmaxf(mx[2], mx[3])) * c;
         const bool move = (mt > m + kRescaleThreshold) || (m == -INFINITY && mt > -INFINITY);
         float alpha = 1.f;
         if (move) {
@@ -367,6 +380,11 @@ __global__ void __launch_bounds__(384, 1)
           if constexpr (PTM) {
             // keys 32cc..32cc+31 -> columns 16cc..16cc+15 of this row's S block
             tmem_st16(tS + 16 * cc, pk);
+            if (cc == 1) {  // first 64 keys of P are in place
+              tmem_wait_st();
+              tc_fence_before();
+              mbar_arrive(bar(C::BAR_P + 2 * k));
+            }
           } else {
             // keys 32cc..32cc+31 -> 64-key region cc/2, 16-byte chunks (cc&1)*4 + 0..3
             const uint32_t region = pbase + (cc >> 1) * 16384;
@@ -383,7 +401,8 @@ __global__ void __launch_bounds__(384, 1)
           fence_proxy_async_smem();
         }
         tc_fence_before();
-        mbar_arrive(bar(C::BAR_P + k));
+        if constexpr (!PTM) mbar_arrive(bar(C::BAR_P + 2 * k));
+        mbar_arrive(bar(C::BAR_P + 2 * k + 1));
       }
       if (ok) {
         ok = mbar_wait(bar(C::BAR_S + k), nk & 1, abort_flag);
