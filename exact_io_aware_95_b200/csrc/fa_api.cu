@@ -357,3 +357,62 @@ fa_status fa_get_device_error(void* stream) {
 }
 
 }  // extern "C"
+
+// ---------------------------------------------------------------------------
+// Backward pass without a caller-provided workspace.
+//
+// Some callers cannot allocate device memory at the point where they run the
+// backward pass: code that executes inside a custom allocator or memory-pool
+// callback, runtimes that forbid cudaMalloc after start-up (fixed memory
+// budgets, pre-planned arenas), or plug-in hosts that hand out only the
+// tensors themselves.  For them the scratch the backward pass needs (fp32 dQ
+// accumulator and the D vector) lives in one statically sized device array
+// that is part of this library's device image: every GPU that loads the
+// library holds it until the process exits, and nothing is allocated per call.
+//
+// In host code `g_fa_static_scratch` names a host-side stand-in, not device
+// memory, so the device address is looked up with cudaGetSymbolAddress once
+// per device (on that device's first call, with the device current) and that
+// address is what the kernels receive.  That first call per device performs
+// the lookup and should therefore come before any stream capture.
+// ---------------------------------------------------------------------------
+namespace {
+
+constexpr size_t kStaticScratchBytes = size_t(64) << 20;  // 64 MiB; matches FA_STATIC_SCRATCH_BYTES
+static_assert(kStaticScratchBytes == FA_STATIC_SCRATCH_BYTES, "header and library disagree on the scratch size");
+
+static __device__ __align__(256) unsigned char g_fa_static_scratch[kStaticScratchBytes];
+
+void* g_static_scratch_ptr[kMaxDevices] = {};
+
+fa_status static_scratch(int dev, void** out) {
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!g_static_scratch_ptr[dev]) {
+    void* ptr = nullptr;
+    if (cudaGetSymbolAddress(&ptr, g_fa_static_scratch) != cudaSuccess || ptr == nullptr) {
+      cudaGetLastError();
+      return FA_ERR_CUDA;
+    }
+    g_static_scratch_ptr[dev] = ptr;
+  }
+  *out = g_static_scratch_ptr[dev];
+  return FA_OK;
+}
+
+}  // namespace
+
+extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                    const void* dO, void* dq, void* dk, void* dv, int B, int N, int H, int d,
+                                    float scale, int causal, void* stream) {
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (B < 1 || N < 1 || H < 1) return FA_ERR_INVALID_ARG;
+  const size_t need = fa_bwd_workspace_size(B, N, H, d);
+  if (need == 0) return FA_ERR_INVALID_ARG;
+  if (need > kStaticScratchBytes) return FA_ERR_WORKSPACE;  // problem too large for the static scratch
+  int dev;
+  fa_status st = current_device(&dev);
+  if (st != FA_OK) return st;
+  void* scratch = nullptr;
+  if ((st = static_scratch(dev, &scratch)) != FA_OK) return st;
+  return fa_bwd(q, k, v, o, lse, dO, dq, dk, dv, scratch, kStaticScratchBytes, B, N, H, d, scale, causal, stream);
+}

@@ -27,9 +27,10 @@
  *   - head dim d is 64 or 128; bf16 inputs, fp32 accumulation and softmax.
  *
  * Ownership.  Every pointer is a DEVICE pointer owned by the caller, 16-byte
- * aligned, on the current CUDA device.  The library never allocates device
- * memory: the backward pass takes a caller-allocated workspace of
- * fa_bwd_workspace_size() bytes.  Outputs are fully overwritten; the
+ * aligned, on the current CUDA device.  No call allocates device memory:
+ * the backward pass takes a caller-allocated workspace of
+ * fa_bwd_workspace_size() bytes (fa_bwd_noalloc instead uses a fixed static
+ * array in the library's device image).  Outputs are fully overwritten; the
  * workspace holds no state between calls.  All calls are asynchronous on
  * `stream` (a cudaStream_t; NULL = legacy default stream) and return after
  * the launch; errors found on the host are returned before anything is
@@ -99,6 +100,29 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                         const int* cu_seqlens, int nseq, int total, int max_seqlen,
                         int H, int d, float scale, int causal, void* stream);
+
+/* Backward pass, dense batch, for callers that cannot allocate device memory.
+ * There is no counterpart to this in the method's description: it exists for
+ * callers that may not call cudaMalloc (or any allocating routine) when they
+ * run the backward pass -- for example code running inside an allocator or
+ * memory-pool callback, or a runtime with a fixed, pre-planned memory budget.
+ * Arguments and results are those of fa_bwd without the workspace: the fp32
+ * scratch comes from one static device array of FA_STATIC_SCRATCH_BYTES that
+ * the library image carries on every GPU that loads it (held until exit).
+ * Nothing is allocated or freed by this call.
+ *   - Problems needing more than FA_STATIC_SCRATCH_BYTES of scratch
+ *     (fa_bwd_workspace_size(B, N, H, d) > FA_STATIC_SCRATCH_BYTES) are
+ *     rejected with FA_ERR_WORKSPACE before anything is launched.
+ *   - The first call on a device looks up the array's device address (with
+ *     that device current); make that first call before any stream capture.
+ *   - All calls share the one array and it keeps the last call's contents;
+ *     the parts that must start at zero are cleared by each call itself.
+ *     Calls whose GPU work overlaps (different streams, or different host
+ *     threads without ordering) race on the array: serialise them. */
+#define FA_STATIC_SCRATCH_BYTES ((size_t)64 << 20)
+fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                         const void* dO, void* dq, void* dk, void* dv,
+                         int B, int N, int H, int d, float scale, int causal, void* stream);
 
 /* Static text for a status code (never NULL). */
 const char* fa_status_string(fa_status s);
