@@ -192,6 +192,12 @@ def barrier(world):
         dist.barrier()
 
 
+def aggregate_tflops(flops_per_rank_step: float, world: int, ms_per_step_max: float) -> float:
+    """Whole-job throughput: the work all ranks did per step over the slowest
+    rank's step time (weak scaling: every rank runs its own shard of equal size)."""
+    return flops_per_rank_step * world / (ms_per_step_max * 1e-3) / 1e12
+
+
 def allmax(x: float, world: int) -> float:
     if world == 1:
         return x
@@ -275,7 +281,7 @@ def run_gpu(args, world, rank, local):
 
     ff = fwd_flops(B, N, H, d, causal)
     bf = 2.5 * ff
-    value = (ff + bf) * world / (ms_step * 1e-3) / 1e12
+    value = aggregate_tflops(ff + bf, world, ms_step)
     fwd_tflops = ff / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = bf / (bwd_ms * 1e-3) / 1e12
     peaks = load_peaks()
@@ -308,7 +314,7 @@ def run_gpu(args, world, rank, local):
     torch.cuda.synchronize(dev)
     barrier(world)
     e2e_ms = allmax(s0.elapsed_time(s1), world) / e_steps
-    e2e_value = (ff + bf) * world / (e2e_ms * 1e-3) / 1e12
+    e2e_value = aggregate_tflops(ff + bf, world, e2e_ms)
 
     if rank != 0:
         return None
@@ -325,7 +331,8 @@ def run_gpu(args, world, rank, local):
                          "fwd_vs_burst": fwd_tflops / peaks["bf16_tflops"],
                          "bwd_vs_burst": bwd_tflops / peaks["bf16_tflops"],
                          "peak_source": peaks["source"]},
-        "roofline": {"kernel": "fa_bwd call (preprocess + main + dq_convert launches)", "bound": "tensor",
+        "roofline": {"kernel": "fa_bwd_kernel (timed as the whole fa_bwd call: preprocess + main + dq_convert)",
+                     "bound": "tensor",
                      "achieved": bwd_tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
                      "frac": bwd_tflops / peaks["bf16_tflops_sustained"],
                      "peak_kind": f"sustained bf16 GEMM ({peaks['source']})",
