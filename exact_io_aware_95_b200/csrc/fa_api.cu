@@ -71,9 +71,9 @@ fa_status current_device(int* dev) {
 
 // Set the dynamic shared-memory limit of `kern` once per device.  Kernels
 // that re-balance registers between warpgroups (setmaxnreg) must have been
-// compiled to exactly fa::kLaunchRegs registers per thread: their split adds
-// up to 384 * kLaunchRegs, and a split larger than the launch allocation
-// would never be granted.  Refuse to launch such a kernel otherwise.
+// compiled to exactly the register count their split was planned for (the
+// split adds up to the launch allocation; a larger one would never be
+// granted).  Refuse to launch such a kernel otherwise.
 template <typename K>
 fa_status ensure_smem(K kern, int dev, int bytes, bool* done_flags, int need_regs = 0) {
   std::lock_guard<std::mutex> lk(g_mu);
@@ -202,7 +202,7 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   static bool done[kMaxDevices] = {};
   auto kern = fa::fa_bwd_kernel<D, CAUSAL, VARLEN>;
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
-  fa_status st = ensure_smem(kern, dev, smem, done, fa::kLaunchRegs);
+  fa_status st = ensure_smem(kern, dev, smem, done, fa::BwdCfg<D>::LAUNCH_REGS);
   if (st != FA_OK) return st;
   // 1) D = rowsum(dO * O) and zeroed dQ accumulator
   {

@@ -29,14 +29,16 @@
 // products.  The dQ product reads the same dS^T buffer through an MN-major
 // descriptor, so dS is written once.
 //
-// Warp roles of the main kernel (384 threads, three warpgroups):
-//   warps 0-3  P^T and dS^T (thread t = key row t), final dK/dV stores
-//   warps 4-7  dQ_i drain: tensor memory -> fp32 atomics (thread t = query row t)
-//   warp  8    TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring
-//   warp  9    tensor-memory allocator and the single MMA-issuing thread
-//   warps 10-11 idle
-// Registers: the producer/MMA warpgroup drops to 96, the P/dS warpgroup rises
-// to 224, the drain warpgroup keeps the launch value.
+// Warp roles of the main kernel (512 threads, four warpgroups):
+//   warps 0-7   P^T and dS^T: thread t of warpgroup w owns key row t and query
+//               columns 64w..64w+63 (two warpgroups per row halve the
+//               per-tile latency of the exponentials and of dS^T); final dK
+//               (warpgroup 0) and dV (warpgroup 1) stores
+//   warps 8-11  dQ_i drain: tensor memory -> fp32 atomics (thread t = query row t)
+//   warp  12    TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring
+//   warp  13    tensor-memory allocator and the single MMA-issuing thread
+//   warps 14-15 idle
+// Registers (launch 128 each): P/dS warpgroups 152, drain 104, producer/MMA 104.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -180,17 +182,18 @@ struct BwdCfg {
   static constexpr int NBAR = BAR_DRAIN + 1;
   static constexpr int OFF_MISC = OFF_BAR + NBAR * 8;
   static constexpr int SMEM_BYTES = OFF_MISC + 16 + 1024;
-  // tensor memory: S^T (P^T packed into its first 64 columns) | dP^T | dK | dV  [| dQ]
+  // tensor memory: S^T (P^T packed into columns 0-31 and 64-95) | dP^T | dK | dV  [| dQ]
   static constexpr int TM_S = 0, TM_DP = 128, TM_DK = 256, TM_DV = 256 + D;
   static constexpr bool DQ_ALIASES_DP = (256 + 2 * D + D) > 512;
   static constexpr int TM_DQ = DQ_ALIASES_DP ? TM_DP : 256 + 2 * D;
   static constexpr int TMEM_COLS = 512;
-  static constexpr int THREADS = 384;
+  static constexpr int THREADS = 512;
+  static constexpr int LAUNCH_REGS = 128;  // 65536 / 512; the setmaxnreg split below sums to 4 x 128
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
 template <int D, bool CAUSAL, bool VARLEN>
-__global__ void __launch_bounds__(384, 1)
+__global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
                   const BwdParams p) {
@@ -245,8 +248,8 @@ __global__ void __launch_bounds__(384, 1)
     }
     mbar_init(bar(C::BAR_S), 1);
     mbar_init(bar(C::BAR_DP), 1);
-    mbar_init(bar(C::BAR_P), 128);
-    mbar_init(bar(C::BAR_DS), 128);
+    mbar_init(bar(C::BAR_P), 256);
+    mbar_init(bar(C::BAR_DS), 256);
     mbar_init(bar(C::BAR_DS_EMPTY), 1);
     mbar_init(bar(C::BAR_DQ_FULL), 1);
     mbar_init(bar(C::BAR_DQ_EMPTY), 128);
@@ -255,7 +258,7 @@ __global__ void __launch_bounds__(384, 1)
     *abort_flag = 0;
     fence_mbar_init();
   }
-  if (warp == 9) {
+  if (warp == 13) {
     tmem_alloc(smem_u32(tmem_slot), C::TMEM_COLS);
     tmem_relinquish();
   }
@@ -263,10 +266,10 @@ __global__ void __launch_bounds__(384, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
-  if (warp >= 8) {
-    regs_dec<96>();
+  if (warp >= 12) {
+    regs_dec<104>();
   }
-  if (warp == 8) {
+  if (warp == 12) {
     // ------------------------------------------------------------ producer
     if (lane == 0) {
       tma_prefetch_desc(&tmQ);
@@ -302,19 +305,29 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     __syncwarp();
-  } else if (warp == 9) {
+  } else if (warp == 13) {
     // ------------------------------------------------------------ MMA issuer
     if (lane == 0) {
       constexpr uint32_t kIdSq = idesc_bf16_f32(128, 128, false, false);  // S^T, dP^T
       constexpr uint32_t kIdDV = idesc_bf16_f32(128, D, false, true);     // dV (A in TMEM), dK
       constexpr uint32_t kIdDQ = idesc_bf16_f32(128, D, true, true);      // dQ: A = dS (MN-major view)
+      // operand descriptors, built once; per MMA only the start address moves
+      const uint64_t dK_k = sdesc_sw128(sbase + C::OFF_K, 16, 1024);        // K as K-major A of S^T
+      const uint64_t dV_k = sdesc_sw128(sbase + C::OFF_V, 16, 1024);        // V as K-major A of dP^T
+      const uint64_t dK_mn = sdesc_sw128(sbase + C::OFF_K, 16384, 1024);    // K as MN-major B of dQ
+      const uint64_t dS_k = sdesc_sw128(sbase + C::OFF_DS, 16, 1024);       // dS^T as K-major A of dK
+      const uint64_t dS_mn = sdesc_sw128(sbase + C::OFF_DS, 16384, 1024);   // dS as MN-major A of dQ
+      const uint64_t dQ0_k = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);       // Q stage 0, K-major B of S^T
+      const uint64_t dQ0_mn = sdesc_sw128(sbase + C::OFF_Q, 16384, 1024);   // Q stage 0, MN-major B of dK
+      const uint64_t dO0_k = sdesc_sw128(sbase + C::OFF_DO, 16, 1024);      // dO stage 0, K-major B of dP^T
+      const uint64_t dO0_mn = sdesc_sw128(sbase + C::OFF_DO, 16384, 1024);  // dO stage 0, MN-major B of dV
+      constexpr uint32_t kStageAdv = C::TILE_BYTES >> 4;
       auto issue_s = [&](int it) {  // S^T = K Q_it^T
-        const uint32_t sQ = sbase + C::OFF_Q + (it % C::NSTAGE) * C::TILE_BYTES;
+        const uint64_t bq = dQ0_k + (it % C::NSTAGE) * kStageAdv;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S, sdesc_sw128(sbase + C::OFF_K + off, 16, 1024), sdesc_sw128(sQ + off, 16, 1024),
-                  kIdSq, kk > 0);
+          umma_ss(tmem + C::TM_S, sdesc_adv(dK_k, off), sdesc_adv(bq, off), kIdSq, kk > 0);
         }
         umma_commit(bar(C::BAR_S));
       };
@@ -329,14 +342,16 @@ __global__ void __launch_bounds__(384, 1)
       for (int it = 0; ok && it < niter; ++it) {
         const int st = it % C::NSTAGE;
         const uint32_t par = it & 1;
-        const uint32_t sQ = sbase + C::OFF_Q + st * C::TILE_BYTES;
-        const uint32_t sdO = sbase + C::OFF_DO + st * C::TILE_BYTES;
+        const uint64_t q_mn = dQ0_mn + st * kStageAdv;
+        const uint64_t o_k = dO0_k + st * kStageAdv;
+        const uint64_t o_mn = dO0_mn + st * kStageAdv;
         // dV += P^T dO   (A = P^T packed bf16 in tensor memory)
         if (!(ok = mbar_wait(bar(C::BAR_P), par, abort_flag))) break;
         tc_fence_after();
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8, sdesc_sw128(sdO + kk * 2048, 16384, 1024), kIdDV,
+          // queries 16kk..16kk+15 of P^T: columns 8kk (first 64 queries) or 32 + 8kk (last 64)
+          umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8 + (kk >= 4 ? 32 : 0), sdesc_adv(o_mn, kk * 2048), kIdDV,
                   (it > 0 || kk > 0));
         // dP^T = V dO^T  (its columns may hold the previous dQ tile: wait until drained)
         if (C::DQ_ALIASES_DP && it > 0) {
@@ -346,8 +361,7 @@ __global__ void __launch_bounds__(384, 1)
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
           const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP, sdesc_sw128(sbase + C::OFF_V + off, 16, 1024), sdesc_sw128(sdO + off, 16, 1024),
-                  kIdSq, kk > 0);
+          umma_ss(tmem + C::TM_DP, sdesc_adv(dV_k, off), sdesc_adv(o_k, off), kIdSq, kk > 0);
         }
         umma_commit(bar(C::BAR_DP));
         // S^T of the next query tile (P^T(i) was consumed by dV above, in issue order)
@@ -360,19 +374,17 @@ __global__ void __launch_bounds__(384, 1)
         // dK += dS^T Q ;  dQ_i = dS K
         if (!(ok = mbar_wait(bar(C::BAR_DS), par, abort_flag))) break;
         tc_fence_after();
-        const uint32_t sDS = sbase + C::OFF_DS;
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + C::TM_DK, sdesc_sw128(sDS + (kk >> 2) * 16384 + (kk & 3) * 32, 16, 1024),
-                  sdesc_sw128(sQ + kk * 2048, 16384, 1024), kIdDV, (it > 0 || kk > 0));
+          umma_ss(tmem + C::TM_DK, sdesc_adv(dS_k, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_adv(q_mn, kk * 2048), kIdDV,
+                  (it > 0 || kk > 0));
         if (!C::DQ_ALIASES_DP && it > 0) {
           if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
           tc_fence_after();
         }
 #pragma unroll
         for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + C::TM_DQ, sdesc_sw128(sDS + kk * 2048, 16384, 1024),
-                  sdesc_sw128(sbase + C::OFF_K + kk * 2048, 16384, 1024), kIdDQ, kk > 0);
+          umma_ss(tmem + C::TM_DQ, sdesc_adv(dS_mn, kk * 2048), sdesc_adv(dK_mn, kk * 2048), kIdDQ, kk > 0);
         umma_commit(bar(C::BAR_QDO_EMPTY + st));
         umma_commit(bar(C::BAR_DS_EMPTY));
         umma_commit(bar(C::BAR_DQ_FULL));
@@ -384,25 +396,27 @@ __global__ void __launch_bounds__(384, 1)
       }
     }
     __syncwarp();
-  } else if (warp < 4) {
+  } else if (warp < 8) {
     // ------------------------------------------------------------ P^T and dS^T
-    regs_inc<224>();
-    const int t = threadIdx.x;  // key row within the tile == tensor-memory lane
+    regs_inc<152>();
+    const int w = warp >> 2;          // this warpgroup's query columns: 64w .. 64w+63
+    const int t = threadIdx.x & 127;  // key row within the tile == tensor-memory lane
     const int key = k0 + t;
     const bool key_ok = key < L;
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>(warp * 32) << 16);
+    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     float* sLSE = reinterpret_cast<float*>(smem + C::OFF_LSE);
     float* sDv = reinterpret_cast<float*>(smem + C::OFF_DV);
     const float c = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     bool ok = true;
-    // LSE (base 2) and D of query row q of the tile starting at q0; rows past
-    // the sequence get LSE = +inf so their P is exactly 0.
+    // LSE (base 2) and D of this warpgroup's query columns: thread t < 64
+    // fetches column 64w + t of the tile starting at q0.  Rows past the
+    // sequence get LSE = +inf so their P is exactly 0.
     auto fetch = [&](int q0, float& lv, float& dv) {
-      const int q = q0 + t;
+      const int q = q0 + 64 * w + t;
       lv = INFINITY;
       dv = 0.f;
-      if (q < L) {
+      if (t < 64 && q < L) {
         const size_t li = VARLEN ? (static_cast<size_t>(h) * p.total + tok0 + q)
                                  : ((static_cast<size_t>(b) * p.H + h) * p.N + q);
         lv = p.lse[li] * kLog2e;
@@ -414,10 +428,12 @@ __global__ void __launch_bounds__(384, 1)
     for (int it = 0; it < niter; ++it) {
       const uint32_t par = it & 1;
       const int q0 = 128 * (i_begin + it);
-      named_bar_sync(1, 128);  // everyone is done with the previous tile's values
-      sLSE[t] = lv_next;
-      sDv[t] = dv_next;
-      named_bar_sync(1, 128);
+      named_bar_sync(1 + w, 128);  // the warpgroup is done with the previous tile's values
+      if (t < 64) {
+        sLSE[64 * w + t] = lv_next;
+        sDv[64 * w + t] = dv_next;
+      }
+      named_bar_sync(1 + w, 128);
       if (it + 1 < niter) fetch(q0 + 128, lv_next, dv_next);  // lands during this tile
       ok = mbar_wait(bar(C::BAR_S), par, abort_flag);
       if (!__all_sync(0xffffffffu, ok)) {
@@ -427,9 +443,10 @@ __global__ void __launch_bounds__(384, 1)
       tc_fence_after();
       const bool diag = CAUSAL && (q0 == k0);
       const float4* sLSE4 = reinterpret_cast<const float4*>(sLSE);
-      uint32_t pk[4][16];
+      uint32_t pk[2][16];
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int hc = 0; hc < 2; ++hc) {
+        const int cc = 2 * w + hc;  // 32-column chunk of the 128-column tile
         uint32_t s[32];
         tmem_ld32(lane_base + C::TM_S + 32 * cc, s);
         tmem_wait_ld(s);
@@ -448,14 +465,15 @@ __global__ void __launch_bounds__(384, 1)
             if (t > qa + 3) p3 = 0.f;
           }
           if (!key_ok) p0 = p1 = p2 = p3 = 0.f;
-          pk[cc][2 * m] = pack_bf16x2(p0, p1);
-          pk[cc][2 * m + 1] = pack_bf16x2(p2, p3);
+          pk[hc][2 * m] = pack_bf16x2(p0, p1);
+          pk[hc][2 * m + 1] = pack_bf16x2(p2, p3);
         }
+        // P^T (bf16) is packed into the first half of this warpgroup's own
+        // S^T columns: query chunk cc = 2w + hc -> columns 64w + 16hc .. +15.
+        // This thread has already loaded those S^T values (its own lane), and
+        // the other warpgroup never touches these columns.
+        tmem_st16(lane_base + C::TM_S + 64 * w + 16 * hc, pk[hc]);
       }
-      // P^T (bf16) into the first 64 columns of the S^T block; every S^T value
-      // has been read above
-#pragma unroll
-      for (int cc = 0; cc < 4; ++cc) tmem_st16(lane_base + C::TM_S + 16 * cc, pk[cc]);
       tmem_wait_st();
       tc_fence_before();
       mbar_arrive(bar(C::BAR_P));
@@ -466,68 +484,64 @@ __global__ void __launch_bounds__(384, 1)
         break;
       }
       tc_fence_after();
-      const uint32_t sDS = sbase + C::OFF_DS;
+      const uint32_t region = sbase + C::OFF_DS + w * 16384;  // queries 64w..64w+63
+      const float4* sDv4 = reinterpret_cast<const float4*>(sDv);
 #pragma unroll
-      for (int cc = 0; cc < 4; ++cc) {
+      for (int hc = 0; hc < 2; ++hc) {
+        const int cc = 2 * w + hc;
         uint32_t dp[32];
         tmem_ld32(lane_base + C::TM_DP + 32 * cc, dp);
         tmem_wait_ld(dp);
-        const float4* sDv4 = reinterpret_cast<const float4*>(sDv);
-        uint32_t w[16];
+        uint32_t wv[16];
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
           const float4 d4 = sDv4[8 * cc + m];
-          const uint32_t a0 = pk[cc][2 * m], a1 = pk[cc][2 * m + 1];
+          const uint32_t a0 = pk[hc][2 * m], a1 = pk[hc][2 * m + 1];
           const float d0 = bf16lo_to_f32(a0) * (__uint_as_float(dp[4 * m + 0]) - d4.x);
           const float d1 = bf16hi_to_f32(a0) * (__uint_as_float(dp[4 * m + 1]) - d4.y);
           const float d2 = bf16lo_to_f32(a1) * (__uint_as_float(dp[4 * m + 2]) - d4.z);
           const float d3 = bf16hi_to_f32(a1) * (__uint_as_float(dp[4 * m + 3]) - d4.w);
-          w[2 * m] = pack_bf16x2(d0, d1);
-          w[2 * m + 1] = pack_bf16x2(d2, d3);
+          wv[2 * m] = pack_bf16x2(d0, d1);
+          wv[2 * m + 1] = pack_bf16x2(d2, d3);
         }
-        // queries 32cc..32cc+31 -> 64-query region cc/2, 16-byte chunks (cc&1)*4 + 0..3
-        const uint32_t region = sDS + (cc >> 1) * 16384;
+        // 32 queries -> 16-byte chunks hc*4 + 0..3 of this row in region w
 #pragma unroll
         for (int u = 0; u < 4; ++u)
-          st_shared_v4(region + sw128_offset(t, (cc & 1) * 4 + u), w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
+          st_shared_v4(region + sw128_offset(t, hc * 4 + u), wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
       }
       fence_proxy_async_smem();
       tc_fence_before();
       mbar_arrive(bar(C::BAR_DS));
     }
-    // final dK, dV rows
+    // final rows: warpgroup 0 stores dK (times scale), warpgroup 1 stores dV
     if (ok) {
       ok = mbar_wait(bar(C::BAR_ACC), 0, abort_flag);
       if (__all_sync(0xffffffffu, ok)) {
         tc_fence_after();
         const size_t row = ((VARLEN ? static_cast<size_t>(tok0) : static_cast<size_t>(b) * p.N) + key) * p.H + h;
-        __nv_bfloat16* dkrow = reinterpret_cast<__nv_bfloat16*>(p.dk) + row * D;
-        __nv_bfloat16* dvrow = reinterpret_cast<__nv_bfloat16*>(p.dv) + row * D;
+        const uint32_t col = w ? C::TM_DV : C::TM_DK;
+        const float mul = w ? 1.f : p.scale;
+        __nv_bfloat16* dst = reinterpret_cast<__nv_bfloat16*>(w ? p.dv : p.dk) + row * D;
 #pragma unroll 1
-        for (int which = 0; which < 2; ++which) {
-          const uint32_t col = which ? C::TM_DV : C::TM_DK;
-          const float mul = which ? 1.f : p.scale;
-          __nv_bfloat16* dst = which ? dvrow : dkrow;
-#pragma unroll 1
-          for (int cc = 0; cc < D / 32; ++cc) {
-            uint32_t a[32];
-            tmem_ld32(lane_base + col + 32 * cc, a);
-            tmem_wait_ld(a);
-            uint32_t w[16];
+        for (int cc = 0; cc < D / 32; ++cc) {
+          uint32_t a[32];
+          tmem_ld32(lane_base + col + 32 * cc, a);
+          tmem_wait_ld(a);
+          uint32_t wv[16];
 #pragma unroll
-            for (int i = 0; i < 16; ++i)
-              w[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
-            if (key_ok) {
+          for (int i = 0; i < 16; ++i)
+            wv[i] = pack_bf16x2(__uint_as_float(a[2 * i]) * mul, __uint_as_float(a[2 * i + 1]) * mul);
+          if (key_ok) {
 #pragma unroll
-              for (int u = 0; u < 4; ++u) st_global_v4(dst + 32 * cc + 8 * u, w[4 * u], w[4 * u + 1], w[4 * u + 2], w[4 * u + 3]);
-            }
+            for (int u = 0; u < 4; ++u) st_global_v4(dst + 32 * cc + 8 * u, wv[4 * u], wv[4 * u + 1], wv[4 * u + 2], wv[4 * u + 3]);
           }
         }
       }
     }
-  } else if (warp < 8) {
+  } else if (warp < 12) {
     // ------------------------------------------------------------ dQ_i drain
-    const int t = threadIdx.x - 128;  // query row within the tile == tensor-memory lane
+    regs_dec<104>();
+    const int t = threadIdx.x - 256;  // query row within the tile == tensor-memory lane
     const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
     for (int it = 0; it < niter; ++it) {
       const uint32_t par = it & 1;
@@ -536,31 +550,39 @@ __global__ void __launch_bounds__(384, 1)
       if (!__all_sync(0xffffffffu, ok)) break;
       tc_fence_after();
       // accumulator rows: (bh, float4 group g, r) with r consecutive across the warp
-      const int bh = VARLEN ? h : b * p.H + h;
+      const int bh_ = VARLEN ? h : b * p.H + h;
       const int64_t R = VARLEN ? p.total : p.N;
       const int64_t r = static_cast<int64_t>(VARLEN ? tok0 : 0) + q;
       float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
+      // 64 columns at a time; the tile's columns are released once the last
+      // load has landed (the atomics then run from registers)
 #pragma unroll 1
-      for (int cc = 0; cc < D / 32; ++cc) {
-        uint32_t a[32];
-        tmem_ld32(lane_base + C::TM_DQ + 32 * cc, a);
-        tmem_wait_ld(a);
+      for (int cg = 0; cg < D / 32; cg += 2) {
+        uint32_t a[2][32];
+        tmem_ld32(lane_base + C::TM_DQ + 32 * cg, a[0]);
+        tmem_ld32(lane_base + C::TM_DQ + 32 * (cg + 1), a[1]);
+        tmem_wait_ld(a[0]);
+        tmem_wait_ld(a[1]);
+        if (cg + 2 >= D / 32) {
+          tc_fence_before();
+          mbar_arrive(bar(C::BAR_DQ_EMPTY));
+        }
         if (q < L) {
 #pragma unroll
-          for (int u = 0; u < 8; ++u)
-            atomicAdd(acc4 + dq_acc_index4(bh, 8 * cc + u, r, R, D),
-                      make_float4(__uint_as_float(a[4 * u]), __uint_as_float(a[4 * u + 1]),
-                                  __uint_as_float(a[4 * u + 2]), __uint_as_float(a[4 * u + 3])));
+          for (int e = 0; e < 2; ++e)
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              atomicAdd(acc4 + dq_acc_index4(bh_, 8 * (cg + e) + u, r, R, D),
+                        make_float4(__uint_as_float(a[e][4 * u]), __uint_as_float(a[e][4 * u + 1]),
+                                    __uint_as_float(a[e][4 * u + 2]), __uint_as_float(a[e][4 * u + 3])));
         }
       }
-      tc_fence_before();
-      mbar_arrive(bar(C::BAR_DQ_EMPTY));
     }
   }
 
   tc_fence_before();
   __syncthreads();
-  if (warp == 9) {
+  if (warp == 13) {
     tc_fence_after();
     tmem_dealloc(tmem, C::TMEM_COLS);
   }

@@ -21,8 +21,8 @@
 //   warp  8    TMA producer: Q0, Q1 once, then K_j, V_j into an NSTAGE ring
 //   warp  9    tensor-memory allocator and the single MMA-issuing thread
 //   warps 10-11 idle
-// The producer/MMA warpgroup gives up registers (56 each) so the two softmax
-// warpgroups can hold a whole 128-column score row (224 each).
+// The producer/MMA warpgroup gives up registers (72 each) so the two softmax
+// warpgroups can hold a whole 128-column score row (216 each).
 // The split of the non-matmul work into its own warps, so the MMA unit never
 // waits on it more than necessary, is the B200 form of "FlashAttention-2
 // (PT)", sections "1. Minimizacao de operacoes nao matriciais" and "3. Divisao
@@ -165,7 +165,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
-    regs_dec<56>();
+    regs_dec<72>();
   }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -210,24 +210,30 @@ __global__ void __launch_bounds__(384, 1)
     if (lane == 0) {
       constexpr uint32_t kIdS = idesc_bf16_f32(128, 128, false, false);
       constexpr uint32_t kIdO = idesc_bf16_f32(128, D, false, true);
+      // operand descriptors, built once; per MMA only the start address moves
+      const uint64_t dQ_k = sdesc_sw128(sbase + C::OFF_Q, 16, 1024);       // Q tiles (K-major A of S)
+      const uint64_t dKV_k = sdesc_sw128(sbase + C::OFF_KV, 16, 1024);     // K stages (K-major B of S)
+      const uint64_t dKV_mn = sdesc_sw128(sbase + C::OFF_KV, 16384, 1024); // V stages (MN-major B of PV)
+      constexpr uint32_t kTileAdv = C::TILE_BYTES >> 4;
       auto issue_s = [&](int k, int st) {
+        const uint64_t a0 = dQ_k + k * kTileAdv;
+        const uint64_t b0 = dKV_k + st * kTileAdv;
 #pragma unroll
         for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t a = sbase + C::OFF_Q + k * C::TILE_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-          const uint32_t bb = sbase + C::OFF_KV + st * C::TILE_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_S + 128 * k, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16, 1024), kIdS, kk > 0);
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_S + 128 * k, sdesc_adv(a0, off), sdesc_adv(b0, off), kIdS, kk > 0);
         }
       };
       auto issue_pv = [&](int k, int st, int j, int kk0) {
+        const uint64_t b0 = dKV_mn + st * kTileAdv;
 #pragma unroll
         for (int kk = kk0; kk < kk0 + 4; ++kk) {
-          const uint32_t bb = sbase + C::OFF_KV + st * C::TILE_BYTES + kk * 2048;
           if constexpr (PTM) {
-            umma_ts(tmem + C::TM_O + D * k, tmem + C::TM_S + 128 * k + kk * 8, sdesc_sw128(bb, 16384, 1024), kIdO,
+            umma_ts(tmem + C::TM_O + D * k, tmem + C::TM_S + 128 * k + kk * 8, sdesc_adv(b0, kk * 2048), kIdO,
                     (j > 0 || kk > 0));
           } else {
             const uint32_t a = sbase + C::OFF_P + k * C::P_BYTES + (kk >> 2) * 16384 + (kk & 3) * 32;
-            umma_ss(tmem + C::TM_O + D * k, sdesc_sw128(a, 16, 1024), sdesc_sw128(bb, 16384, 1024), kIdO,
+            umma_ss(tmem + C::TM_O + D * k, sdesc_sw128(a, 16, 1024), sdesc_adv(b0, kk * 2048), kIdO,
                     (j > 0 || kk > 0));
           }
         }
@@ -298,7 +304,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
-    regs_inc<224>();
+    regs_inc<216>();
     const int k = warp >> 2;
     const int t = threadIdx.x & 127;  // row within the query tile == tensor-memory lane
     const int nk = ntile[k];

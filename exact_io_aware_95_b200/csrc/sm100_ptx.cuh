@@ -161,6 +161,15 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
   return d;
 }
 
+// Advance a descriptor within its operand tile: the start address sits in the
+// low 14 bits as (address >> 4), so a byte offset is added as (offset >> 4).
+// Every tile lies below 256 KiB of shared memory, so the field never carries
+// into the leading-offset bits.  One integer add per MMA keeps the single
+// issuing thread far ahead of the tensor core.
+__device__ __forceinline__ uint64_t sdesc_adv(uint64_t desc, uint32_t byte_off) {
+  return desc + static_cast<uint64_t>(byte_off >> 4);
+}
+
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.
 __host__ __device__ constexpr uint32_t idesc_bf16_f32(int M, int N, bool a_mn_major, bool b_mn_major) {
   return (1u << 4)                                   // D format: f32

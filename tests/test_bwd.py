@@ -70,3 +70,18 @@ def test_workspace_too_small_raises():
     with pytest.raises(fa.FaError) as e:
         fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], workspace=ws)
     assert e.value.status == fa.FA_ERR_WORKSPACE
+
+
+@pytest.mark.parametrize("d", [64, 128])
+def test_repeated_runs_all_within_tolerance(d):
+    """Twenty backward passes of one problem: an ordering race between the
+    warp roles would show up as an occasional wrong result."""
+    x = make_dense(2, 600, 2, d, seed=31)
+    g = {k: v.cuda() for k, v in x.items()}
+    o, lse = fa.fwd(g["q"], g["k"], g["v"], causal=True)
+    G = oracle.attn_bwd_ref(*(f64(x[n]) for n in ("q", "k", "v", "do")), scale_of(d), True)
+    for _ in range(20):
+        dq, dk, dv = fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], causal=True)
+        fa.check_device_error()
+        errs = [rel_fro(f64(t), r) for t, r in zip((dq, dk, dv), G)]
+        assert max(errs) <= GRAD_RTOL_FRO, errs
