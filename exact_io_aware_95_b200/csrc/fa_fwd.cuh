@@ -33,9 +33,11 @@
 //
 // Softmax details: scores are handled in base 2 with c = scale*log2(e) folded
 // into one FMA per element.  The reference max m is only moved (and O, l
-// rescaled) when the tile max exceeds it by more than 8 (a factor 256); P
-// entries stay <= 2^8, so fp32/bf16 range is never at risk and the final
-// O/l and LSE = (m + log2 l) ln 2 are the same exact quantities.
+// rescaled) when the tile max exceeds it by more than 16 (a factor 65536).
+// The final O/l and LSE = (m + log2 l) ln 2 do not depend on which reference
+// is used, so this is still exact: P entries stay <= 2^16 (bf16 and fp32
+// carry them with their usual relative precision) and the fp32 sums stay
+// many orders of magnitude below overflow even for N in the millions.
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -86,7 +88,7 @@ struct FwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-constexpr float kRescaleThreshold = 8.0f;  // log2 units
+constexpr float kRescaleThreshold = 16.0f;  // log2 units
 constexpr float kLn2 = 0.693147180559945309f;
 
 template <int D, bool CAUSAL, bool VARLEN, bool PTM>
