@@ -84,6 +84,12 @@ def _stream_ptr(t: torch.Tensor) -> int:
     return torch.cuda.current_stream(t.device).cuda_stream
 
 
+def _on(t: torch.Tensor):
+    """Make the tensors' device current for the call: the library launches on
+    the calling thread's current device and stream."""
+    return torch.cuda.device(t.device)
+
+
 def _need(t: torch.Tensor, name: str, dtype, ndim: int):
     if not isinstance(t, torch.Tensor):
         raise TypeError(f"{name} must be a torch.Tensor")
@@ -95,6 +101,13 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise ValueError(f"{name} must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
+
+
+def _same_device(*ts):
+    dev = ts[0].device
+    for t in ts[1:]:
+        if t.device != dev:
+            raise ValueError(f"all tensors must be on {dev}; got one on {t.device}")
 
 
 def _scale(scale: Optional[float], d: int) -> float:
@@ -117,8 +130,10 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
     _need(o, "out", torch.bfloat16, 4)
     _need(l, "lse", torch.float32, 3)
-    st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, N, H, d,
-                      _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _same_device(q, k, v, o, l)
+    with _on(q):
+        st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, N, H, d,
+                          _scale(scale, d), int(bool(causal)), _stream_ptr(q))
     _check(st, "fa_fwd")
     return o, l
 
@@ -135,9 +150,11 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                      dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
-                      B, N, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _same_device(q, k, v, o, lse, do, ws, dq, dk, dv)
+    with _on(q):
+        st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                          B, N, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
     _check(st, "fa_bwd")
     return dq, dk, dv
 
@@ -152,9 +169,11 @@ def varlen_fwd(q, k, v, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool 
     nseq = cu_seqlens.numel() - 1
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((H, total), dtype=torch.float32, device=q.device) if lse is None else lse
-    st = lib().fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
-                             cu_seqlens.data_ptr(), nseq, total, int(max_seqlen), H, d, _scale(scale, d),
-                             int(bool(causal)), _stream_ptr(q))
+    _same_device(q, k, v, o, l, cu_seqlens)
+    with _on(q):
+        st = lib().fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                 cu_seqlens.data_ptr(), nseq, total, int(max_seqlen), H, d, _scale(scale, d),
+                                 int(bool(causal)), _stream_ptr(q))
     _check(st, "fa_varlen_fwd")
     return o, l
 
@@ -172,10 +191,12 @@ def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, c
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
-    st = lib().fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                             dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
-                             ws.numel() * ws.element_size(), cu_seqlens.data_ptr(), nseq, total, int(max_seqlen),
-                             H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _same_device(q, k, v, o, lse, do, cu_seqlens, ws, dq, dk, dv)
+    with _on(q):
+        st = lib().fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
+                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
+                                 ws.numel() * ws.element_size(), cu_seqlens.data_ptr(), nseq, total, int(max_seqlen),
+                                 H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
     _check(st, "fa_varlen_bwd")
     return dq, dk, dv
 
@@ -184,3 +205,8 @@ def check_device_error(stream: Optional[torch.cuda.Stream] = None):
     """Synchronise the stream and raise if a kernel gave up on a bounded wait."""
     s = (stream or torch.cuda.current_stream()).cuda_stream
     _check(lib().fa_get_device_error(s), "fa_get_device_error")
+
+
+from .autograd import attention, varlen_attention, pack, unpack  # noqa: E402
+
+__all__ += ["attention", "varlen_attention", "pack", "unpack"]

@@ -40,6 +40,40 @@ EncodeTiledFn encode_fn() {
   return fn;
 }
 
+using CtxGetCurrentFn = CUresult (*)(CUcontext*);
+
+CtxGetCurrentFn ctx_get_current_fn() {
+  static CtxGetCurrentFn fn = nullptr;
+  static bool tried = false;
+  std::lock_guard<std::mutex> lk(g_mu);
+  if (!tried) {
+    tried = true;
+    void* ptr = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuCtxGetCurrent", &ptr, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<CtxGetCurrentFn>(ptr);
+  }
+  return fn;
+}
+
+// A host thread that has not yet made any CUDA context current (a new worker
+// thread, e.g. the one torch's autograd engine runs a backward on) gets one
+// lazily from the first runtime call that needs it; the driver's tensor-map
+// encoder, called before any such runtime call, would fail with
+// CUDA_ERROR_INVALID_CONTEXT.  Bind the current device's primary context in
+// that case.  A context the caller made current is left untouched.
+bool bind_context_if_none(int dev) {
+  CtxGetCurrentFn get = ctx_get_current_fn();
+  CUcontext ctx = nullptr;
+  if (get && get(&ctx) == CUDA_SUCCESS && ctx != nullptr) return true;
+  if (cudaSetDevice(dev) != cudaSuccess) {
+    cudaGetLastError();
+    return false;
+  }
+  return true;
+}
+
 constexpr int kMaxDevices = 64;
 
 // Per-device: compute capability check result and the opt-in shared-memory
@@ -55,6 +89,7 @@ fa_status current_device(int* dev) {
     return FA_ERR_CUDA;
   }
   if (*dev < 0 || *dev >= kMaxDevices) return FA_ERR_UNSUPPORTED;
+  if (!bind_context_if_none(*dev)) return FA_ERR_CUDA;
   std::lock_guard<std::mutex> lk(g_mu);
   DeviceState& st = g_dev[*dev];
   if (st.checked == 0) {
