@@ -17,7 +17,10 @@ reasons are sampled with nvidia-smi during the timed region.
 
 Lines printed: one JSON object (rank 0).  `--impl reference` times the fp64
 CPU oracle instead (the slow baseline), on a bounded sample of the same
-workload.
+workload.  `--sweep` instead times every call of every workload the path is
+specified on (one GPU): 10 warm-up calls, then >= 30 calls each bracketed by
+CUDA events, reported as min / median / p90 with one JSON line per
+(workload, mode, direction).
 """
 from __future__ import annotations
 
@@ -38,7 +41,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, make_dense  # noqa: E402
+from workloads import WORKLOADS, make_dense, make_workload  # noqa: E402
 
 WORKLOAD = "fwd_bwd_causal_b4_h16_n4096_d128_qk2x"
 METRIC = "attention TFLOP/s fwd+bwd (bf16), fraction of B200 dense BF16 peak"
@@ -382,6 +385,102 @@ def run_gpu(args, world, rank, local):
     return line
 
 
+DATASHEET_BF16_TFLOPS = 2250.0  # B200 dense bf16, vendor datasheet (context only)
+
+
+def _pct(xs, q):
+    xs = sorted(xs)
+    return xs[min(len(xs) - 1, int(math.ceil(q * len(xs))) - 1)]
+
+
+def run_sweep(args):
+    """Per-call timing of each workload, mode and direction on one GPU."""
+    import exact_io_aware_95_b200 as fa
+
+    dev = torch.device("cuda", 0)
+    torch.cuda.set_device(dev)
+    stream = torch.cuda.current_stream(dev)
+    peaks = load_peaks()
+    iters = max(30, args.calls)
+    # a buffer larger than L2, written between calls for the flushed variant
+    flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
+    names = [args.only] if args.only else list(WORKLOADS)
+    for name in names:
+        w = WORKLOADS[name]
+        x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in make_workload(w, seed=args.seed).items()}
+        scale = 1.0 / math.sqrt(w.d)
+        flush_variants = (False, True) if w.N and w.N <= 128 else (False,)
+        for causal in w.causal:
+            if w.varlen_total:
+                lens = x["lengths"]
+                ff = sum(4.0 * w.H * L * L * w.d for L in lens) / (2 if causal else 1)
+                mx = max(lens)
+
+                def f():
+                    return fa.varlen_fwd(x["q"], x["k"], x["v"], x["cu_seqlens"], mx, causal=causal, scale=scale,
+                                         out=o, lse=lse)
+
+                def b(det=False):
+                    fa.varlen_bwd(x["q"], x["k"], x["v"], o, lse, x["do"], x["cu_seqlens"], mx, causal=causal,
+                                  scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv, deterministic=det)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((w.H, w.varlen_total), dtype=torch.float32, device=dev)
+                ws = torch.empty(fa.workspace_size(1, w.varlen_total, w.H, w.d), dtype=torch.uint8, device=dev)
+                shape = {"total": w.varlen_total, "nseq": len(lens), "H": w.H, "d": w.d, "lengths": lens}
+            else:
+                ff = fwd_flops(w.B, w.N, w.H, w.d, causal)
+
+                def f():
+                    return fa.fwd(x["q"], x["k"], x["v"], causal=causal, scale=scale, out=o, lse=lse)
+
+                def b(det=False):
+                    fa.bwd(x["q"], x["k"], x["v"], o, lse, x["do"], causal=causal, scale=scale, workspace=ws,
+                           dq=dq, dk=dk, dv=dv, deterministic=det)
+                o = torch.empty_like(x["q"])
+                lse = torch.empty((w.B, w.H, w.N), dtype=torch.float32, device=dev)
+                ws = torch.empty(fa.workspace_size(w.B, w.N, w.H, w.d), dtype=torch.uint8, device=dev)
+                shape = {"B": w.B, "N": w.N, "H": w.H, "d": w.d}
+            dq, dk, dv = (torch.empty_like(x["q"]) for _ in range(3))
+            f()
+            # the deterministic backward is credited with the same algorithmic
+            # FLOPs (2.5x forward); its recomputation of S and dP is not counted
+            dirs = [("fwd", f, ff)] + ([("bwd", b, 2.5 * ff), ("bwd_deterministic", lambda: b(True), 2.5 * ff)]
+                                       if w.backward else [])
+            for direction, fn, flops in dirs:
+                for flush in flush_variants:
+                    for _ in range(10):
+                        fn()
+                    fa.check_device_error()
+                    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True))
+                           for _ in range(iters)]
+                    clocks = ClockSampler(0)
+                    torch.cuda.synchronize(dev)
+                    clocks.start()
+                    for e0, e1 in evs:
+                        if flush:
+                            flush_buf.fill_(1)
+                        e0.record(stream)
+                        fn()
+                        e1.record(stream)
+                    torch.cuda.synchronize(dev)
+                    clk = clocks.stop()
+                    fa.check_device_error()
+                    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+                    med = statistics.median(ms)
+                    tf = flops / (med * 1e-3) / 1e12
+                    print(json.dumps({
+                        "sweep": name, "causal": causal, "direction": direction, "calls": iters, "warmup": 10,
+                        "l2": "flushed before each call" if flush else "not flushed",
+                        "shape": shape, "gflop": flops / 1e9,
+                        "ms": {"min": min(ms), "median": med, "p90": _pct(ms, 0.9)},
+                        "tflops_at_median": tf,
+                        "frac": {"measured_burst": tf / peaks["bf16_tflops"],
+                                 "measured_sustained": tf / peaks["bf16_tflops_sustained"],
+                                 "datasheet_2250": tf / DATASHEET_BF16_TFLOPS, "peak_source": peaks["source"]},
+                        "clocks": clk}), flush=True)
+        del x
+
+
 def main():
     ap = argparse.ArgumentParser()
     ap.add_argument("--gpus", type=int, default=1)
@@ -390,7 +489,13 @@ def main():
     ap.add_argument("--seed", type=int, default=0)
     ap.add_argument("--impl", choices=["ours", "reference"], default="ours")
     ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--sweep", action="store_true", help="per-call timing of every workload (one GPU)")
+    ap.add_argument("--only", default=None, help="with --sweep: one workload by name")
+    ap.add_argument("--calls", type=int, default=30, help="with --sweep: timed calls per line (>= 30)")
     args = ap.parse_args()
+    if args.sweep:
+        run_sweep(args)
+        return
     if args.warmup < 3:
         args.warmup = 3
     world, rank, local = dist_setup(args)
