@@ -38,6 +38,9 @@ EXPORTS = {
     "fa_bwd_workspace_size": (_S, [_I, _I, _I, _I]),
     "fa_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
     "fa_varlen_bwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _I, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_bwd_deterministic": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_varlen_bwd_deterministic": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _I, _I, _I, _I, _I, _F, _I,
+                                         _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_P]),
@@ -139,8 +142,11 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
 
 
 def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None,
-        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None):
-    """dQ, dK, dV for dense [B, N, H, d] inputs (o, lse from fwd)."""
+        workspace: Optional[torch.Tensor] = None, dq=None, dk=None, dv=None, deterministic: bool = False):
+    """dQ, dK, dV for dense [B, N, H, d] inputs (o, lse from fwd).
+
+    deterministic=True: bitwise reproducible gradients (fa_bwd_deterministic:
+    dQ summed in a fixed order by a second pass instead of fp32 atomics)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _need(t, n, torch.bfloat16, 4)
     _need(lse, "lse", torch.float32, 3)
@@ -152,10 +158,11 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None
     dv = torch.empty_like(v) if dv is None else dv
     _same_device(q, k, v, o, lse, do, ws, dq, dk, dv)
     with _on(q):
-        st = lib().fa_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
-                          dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
-                          B, N, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
-    _check(st, "fa_bwd")
+        fn = lib().fa_bwd_deterministic if deterministic else lib().fa_bwd
+        st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                B, N, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_bwd_deterministic" if deterministic else "fa_bwd")
     return dq, dk, dv
 
 
@@ -179,7 +186,8 @@ def varlen_fwd(q, k, v, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool 
 
 
 def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = False,
-               scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None):
+               scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, deterministic: bool = False):
+    """Packed backward; deterministic=True as for bwd (fa_varlen_bwd_deterministic)."""
     for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
         _need(t, n, torch.bfloat16, 3)
     _need(lse, "lse", torch.float32, 2)
@@ -193,11 +201,12 @@ def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, c
     dv = torch.empty_like(v) if dv is None else dv
     _same_device(q, k, v, o, lse, do, cu_seqlens, ws, dq, dk, dv)
     with _on(q):
-        st = lib().fa_varlen_bwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(),
-                                 do.data_ptr(), dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(),
-                                 ws.numel() * ws.element_size(), cu_seqlens.data_ptr(), nseq, total, int(max_seqlen),
-                                 H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
-    _check(st, "fa_varlen_bwd")
+        fn = lib().fa_varlen_bwd_deterministic if deterministic else lib().fa_varlen_bwd
+        st = fn(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), lse.data_ptr(), do.data_ptr(),
+                dq.data_ptr(), dk.data_ptr(), dv.data_ptr(), ws.data_ptr(), ws.numel() * ws.element_size(),
+                cu_seqlens.data_ptr(), nseq, total, int(max_seqlen), H, d, _scale(scale, d), int(bool(causal)),
+                _stream_ptr(q))
+    _check(st, "fa_varlen_bwd_deterministic" if deterministic else "fa_varlen_bwd")
     return dq, dk, dv
 
 

@@ -26,46 +26,50 @@ __all__ = ["attention", "varlen_attention", "pack", "unpack"]
 
 class _Attention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, causal: bool, scale: Optional[float]):
+    def forward(ctx, q, k, v, causal: bool, scale: Optional[float], deterministic: bool):
         o, lse = _fwd(q, k, v, causal=causal, scale=scale)
         ctx.save_for_backward(q, k, v, o, lse)
-        ctx.causal, ctx.scale = causal, scale
+        ctx.causal, ctx.scale, ctx.deterministic = causal, scale, deterministic
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse = ctx.saved_tensors
-        dq, dk, dv = _bwd(q, k, v, o, lse, do.contiguous(), causal=ctx.causal, scale=ctx.scale)
-        return dq, dk, dv, None, None
+        dq, dk, dv = _bwd(q, k, v, o, lse, do.contiguous(), causal=ctx.causal, scale=ctx.scale,
+                          deterministic=ctx.deterministic)
+        return dq, dk, dv, None, None, None
 
 
 class _VarlenAttention(torch.autograd.Function):
     @staticmethod
-    def forward(ctx, q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: Optional[float]):
+    def forward(ctx, q, k, v, cu_seqlens, max_seqlen: int, causal: bool, scale: Optional[float],
+                deterministic: bool):
         o, lse = _varlen_fwd(q, k, v, cu_seqlens, max_seqlen, causal=causal, scale=scale)
         ctx.save_for_backward(q, k, v, o, lse, cu_seqlens)
-        ctx.max_seqlen, ctx.causal, ctx.scale = max_seqlen, causal, scale
+        ctx.max_seqlen, ctx.causal, ctx.scale, ctx.deterministic = max_seqlen, causal, scale, deterministic
         return o
 
     @staticmethod
     def backward(ctx, do):
         q, k, v, o, lse, cu = ctx.saved_tensors
         dq, dk, dv = _varlen_bwd(q, k, v, o, lse, do.contiguous(), cu, ctx.max_seqlen, causal=ctx.causal,
-                                 scale=ctx.scale)
-        return dq, dk, dv, None, None, None, None
+                                 scale=ctx.scale, deterministic=ctx.deterministic)
+        return dq, dk, dv, None, None, None, None, None
 
 
 def attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
-              scale: Optional[float] = None) -> torch.Tensor:
-    """Exact attention over dense bf16 [B, N, H, d] tensors; differentiable in q, k, v."""
-    return _Attention.apply(q, k, v, bool(causal), scale)
+              scale: Optional[float] = None, deterministic: bool = False) -> torch.Tensor:
+    """Exact attention over dense bf16 [B, N, H, d] tensors; differentiable in q, k, v.
+    deterministic=True makes the gradients bitwise reproducible."""
+    return _Attention.apply(q, k, v, bool(causal), scale, bool(deterministic))
 
 
 def varlen_attention(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, cu_seqlens: torch.Tensor,
-                     max_seqlen: int, causal: bool = False, scale: Optional[float] = None) -> torch.Tensor:
+                     max_seqlen: int, causal: bool = False, scale: Optional[float] = None,
+                     deterministic: bool = False) -> torch.Tensor:
     """Exact attention over a packed batch ([total, H, d], cu_seqlens int32 on the device);
     every sequence attends only to itself.  Differentiable in q, k, v."""
-    return _VarlenAttention.apply(q, k, v, cu_seqlens, int(max_seqlen), bool(causal), scale)
+    return _VarlenAttention.apply(q, k, v, cu_seqlens, int(max_seqlen), bool(causal), scale, bool(deterministic))
 
 
 def pack(seqs: Sequence[torch.Tensor]) -> Tuple[torch.Tensor, torch.Tensor, int]:

@@ -15,6 +15,7 @@
 #define FA_FWD_P_IN_TMEM 1
 #endif
 #include "fa_bwd.cuh"
+#include "fa_bwd_dq.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -231,11 +232,41 @@ size_t ws_bytes_for(int64_t rows, int H, int d) {
   return align256(static_cast<size_t>(rows) * H * d * sizeof(float)) + align256(static_cast<size_t>(rows) * H * sizeof(float));
 }
 
+// Deterministic order: preprocess (D only), dK/dV kernel without its dQ
+// product, then the dQ pass (fixed summation order, no atomics).
+template <int D, bool CAUSAL, bool VARLEN>
+fa_status launch_bwd_det(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
+                         const CUtensorMap& mdo, fa::BwdParams p, int dq_group, cudaStream_t s) {
+  static bool done_main[kMaxDevices] = {};
+  static bool done_dq[kMaxDevices] = {};
+  auto kmain = fa::fa_bwd_kernel<D, CAUSAL, VARLEN, false>;
+  auto kdq = fa::fa_bwd_dq_kernel<D, CAUSAL, VARLEN>;
+  constexpr int smem_main = fa::BwdCfg<D>::SMEM_BYTES;
+  constexpr int smem_dq = fa::DqCfg<D>::SMEM_BYTES;
+  fa_status st = ensure_smem(kmain, dev, smem_main, done_main, fa::BwdCfg<D>::LAUNCH_REGS);
+  if (st != FA_OK) return st;
+  if ((st = ensure_smem(kdq, dev, smem_dq, done_dq)) != FA_OK) return st;
+  p.dq_acc = nullptr;  // no accumulator: the preprocess computes D only
+  const int64_t grid = static_cast<int64_t>(p.nkvtiles) * p.B * p.H;
+  if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
+  {
+    const int64_t blocks = (static_cast<int64_t>(p.rows) * p.H + 7) / 8;
+    if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    if ((st = launch_status()) != FA_OK) return st;
+  }
+  kmain<<<static_cast<unsigned>(grid), fa::BwdCfg<D>::THREADS, smem_main, s>>>(mq, mk, mv, mdo, p);
+  if ((st = launch_status()) != FA_OK) return st;
+  p.group = dq_group;
+  kdq<<<static_cast<unsigned>(grid), fa::DqCfg<D>::THREADS, smem_dq, s>>>(mq, mk, mv, mdo, p);
+  return launch_status();
+}
+
 template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, const CUtensorMap& mv,
                      const CUtensorMap& mdo, const fa::BwdParams& p, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
-  auto kern = fa::fa_bwd_kernel<D, CAUSAL, VARLEN>;
+  auto kern = fa::fa_bwd_kernel<D, CAUSAL, VARLEN, true>;
   constexpr int smem = fa::BwdCfg<D>::SMEM_BYTES;
   fa_status st = ensure_smem(kern, dev, smem, done, fa::BwdCfg<D>::LAUNCH_REGS);
   if (st != FA_OK) return st;
@@ -267,7 +298,15 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
 
 template <int D>
 fa_status dispatch_bwd(int dev, bool causal, bool varlen, const CUtensorMap& q, const CUtensorMap& k,
-                       const CUtensorMap& v, const CUtensorMap& d_o, const fa::BwdParams& p, cudaStream_t s) {
+                       const CUtensorMap& v, const CUtensorMap& d_o, const fa::BwdParams& p, int dq_group,
+                       bool det, cudaStream_t s) {
+  if (det) {
+    if (varlen)
+      return causal ? launch_bwd_det<D, true, true>(dev, q, k, v, d_o, p, dq_group, s)
+                    : launch_bwd_det<D, false, true>(dev, q, k, v, d_o, p, dq_group, s);
+    return causal ? launch_bwd_det<D, true, false>(dev, q, k, v, d_o, p, dq_group, s)
+                  : launch_bwd_det<D, false, false>(dev, q, k, v, d_o, p, dq_group, s);
+  }
   if (varlen)
     return causal ? launch_bwd<D, true, true>(dev, q, k, v, d_o, p, s) : launch_bwd<D, false, true>(dev, q, k, v, d_o, p, s);
   return causal ? launch_bwd<D, true, false>(dev, q, k, v, d_o, p, s) : launch_bwd<D, false, false>(dev, q, k, v, d_o, p, s);
@@ -275,7 +314,7 @@ fa_status dispatch_bwd(int dev, bool causal, bool varlen, const CUtensorMap& q, 
 
 fa_status bwd_common(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                      void* dq, void* dk, void* dv, void* ws, size_t ws_bytes, const int* cu, int B, int N, int total,
-                     int H, int d, float scale, int causal, void* stream) {
+                     int H, int d, float scale, int causal, void* stream, bool det = false) {
   if (!q || !k || !v || !o || !lse || !dO || !dq || !dk || !dv || !ws) return FA_ERR_INVALID_ARG;
   const void* ptrs[] = {q, k, v, o, lse, dO, dq, dk, dv, ws};
   for (const void* ptr : ptrs)
@@ -318,9 +357,11 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
   p.group = head_group(static_cast<int64_t>(N) * d * (2 + 2 + 4), static_cast<int64_t>(B) * H);  // Q, dO, dQ acc
   p.scale = scale;
   p.scale_log2 = scale * kLog2e;
+  // the dQ pass streams K and V of a head once per query tile
+  const int dq_group = head_group(static_cast<int64_t>(N) * d * 2 * 2, static_cast<int64_t>(B) * H);
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
-  return d == 64 ? dispatch_bwd<64>(dev, causal, varlen, mq, mk, mv, mdo, p, s)
-                 : dispatch_bwd<128>(dev, causal, varlen, mq, mk, mv, mdo, p, s);
+  return d == 64 ? dispatch_bwd<64>(dev, causal, varlen, mq, mk, mv, mdo, p, dq_group, det, s)
+                 : dispatch_bwd<128>(dev, causal, varlen, mq, mk, mv, mdo, p, dq_group, det, s);
 }
 
 bool valid_cu(const int* cu, int nseq, int total, int max_seqlen) {
@@ -362,6 +403,23 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total, H, d,
                     scale, causal, stream);
+}
+
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
+                               int N, int H, int d, float scale, int causal, void* stream) {
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, N, H, d, scale, causal,
+                    stream, true);
+}
+
+fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                                      const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                                      const int* cu_seqlens, int nseq, int total, int max_seqlen, int H, int d,
+                                      float scale, int causal, void* stream) {
+  if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total, H, d,
+                    scale, causal, stream, true);
 }
 
 const char* fa_status_string(fa_status s) {

@@ -24,6 +24,10 @@
 //                   atomics.  dK (times scale) and dV are stored once.
 //   3. dq_convert   dQ = bf16(scale * accumulator).
 //
+// Deterministic variant (DQ = false): the main kernel computes dK and dV only
+// and the dQ pass of fa_bwd_dq.cuh sums dQ in a fixed order; the accumulator
+// is then neither zeroed nor converted.
+//
 // Working with S^T instead of S puts one key per tensor-memory lane, so each
 // thread owns one row of P^T and dS^T: exactly the A operands of the dV and dK
 // products.  The dQ product reads the same dS^T buffer through an MN-major
@@ -82,7 +86,7 @@ template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams p) {
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
   const int64_t nacc4 = static_cast<int64_t>(p.rows) * p.H * (D / 4);
-  if (gtid < nacc4) reinterpret_cast<float4*>(p.dq_acc)[gtid] = make_float4(0.f, 0.f, 0.f, 0.f);
+  if (p.dq_acc && gtid < nacc4) reinterpret_cast<float4*>(p.dq_acc)[gtid] = make_float4(0.f, 0.f, 0.f, 0.f);
   const int64_t w = gtid >> 5;
   const int lane = threadIdx.x & 31;
   const int64_t nrows = static_cast<int64_t>(p.rows) * p.H;
@@ -192,7 +196,9 @@ struct BwdCfg {
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
-template <int D, bool CAUSAL, bool VARLEN>
+// DQ: also form dQ_i = dS K_j per tile and add it into the fp32 accumulator
+// (atomic, order varies); without it the kernel computes dK and dV only.
+template <int D, bool CAUSAL, bool VARLEN, bool DQ>
 __global__ void __launch_bounds__(512, 1)
     fa_bwd_kernel(const __grid_constant__ CUtensorMap tmQ, const __grid_constant__ CUtensorMap tmK,
                   const __grid_constant__ CUtensorMap tmV, const __grid_constant__ CUtensorMap tmdO,
@@ -354,7 +360,7 @@ __global__ void __launch_bounds__(512, 1)
           umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8 + (kk >= 4 ? 32 : 0), sdesc_adv(o_mn, kk * 2048), kIdDV,
                   (it > 0 || kk > 0));
         // dP^T = V dO^T  (its columns may hold the previous dQ tile: wait until drained)
-        if (C::DQ_ALIASES_DP && it > 0) {
+        if (DQ && C::DQ_ALIASES_DP && it > 0) {
           if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
           tc_fence_after();
         }
@@ -378,16 +384,18 @@ __global__ void __launch_bounds__(512, 1)
         for (int kk = 0; kk < 8; ++kk)
           umma_ss(tmem + C::TM_DK, sdesc_adv(dS_k, (kk >> 2) * 16384 + (kk & 3) * 32), sdesc_adv(q_mn, kk * 2048), kIdDV,
                   (it > 0 || kk > 0));
-        if (!C::DQ_ALIASES_DP && it > 0) {
-          if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
-          tc_fence_after();
-        }
+        if constexpr (DQ) {
+          if (!C::DQ_ALIASES_DP && it > 0) {
+            if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
+            tc_fence_after();
+          }
 #pragma unroll
-        for (int kk = 0; kk < 8; ++kk)
-          umma_ss(tmem + C::TM_DQ, sdesc_adv(dS_mn, kk * 2048), sdesc_adv(dK_mn, kk * 2048), kIdDQ, kk > 0);
+          for (int kk = 0; kk < 8; ++kk)
+            umma_ss(tmem + C::TM_DQ, sdesc_adv(dS_mn, kk * 2048), sdesc_adv(dK_mn, kk * 2048), kIdDQ, kk > 0);
+        }
         umma_commit(bar(C::BAR_QDO_EMPTY + st));
         umma_commit(bar(C::BAR_DS_EMPTY));
-        umma_commit(bar(C::BAR_DQ_FULL));
+        if (DQ) umma_commit(bar(C::BAR_DQ_FULL));
       }
       if (ok) umma_commit(bar(C::BAR_ACC));
       if (*abort_flag) {
@@ -541,40 +549,42 @@ __global__ void __launch_bounds__(512, 1)
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ_i drain
     regs_dec<104>();
-    const int t = threadIdx.x - 256;  // query row within the tile == tensor-memory lane
-    const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
-    for (int it = 0; it < niter; ++it) {
-      const uint32_t par = it & 1;
-      const int q = 128 * (i_begin + it) + t;
-      bool ok = mbar_wait(bar(C::BAR_DQ_FULL), par, abort_flag);
-      if (!__all_sync(0xffffffffu, ok)) break;
-      tc_fence_after();
-      // accumulator rows: (bh, float4 group g, r) with r consecutive across the warp
-      const int bh_ = VARLEN ? h : b * p.H + h;
-      const int64_t R = VARLEN ? p.total : p.N;
-      const int64_t r = static_cast<int64_t>(VARLEN ? tok0 : 0) + q;
-      float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
-      // 64 columns at a time; the tile's columns are released once the last
-      // load has landed (the atomics then run from registers)
+    if constexpr (DQ) {
+      const int t = threadIdx.x - 256;  // query row within the tile == tensor-memory lane
+      const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
+      for (int it = 0; it < niter; ++it) {
+        const uint32_t par = it & 1;
+        const int q = 128 * (i_begin + it) + t;
+        bool ok = mbar_wait(bar(C::BAR_DQ_FULL), par, abort_flag);
+        if (!__all_sync(0xffffffffu, ok)) break;
+        tc_fence_after();
+        // accumulator rows: (bh, float4 group g, r) with r consecutive across the warp
+        const int bh_ = VARLEN ? h : b * p.H + h;
+        const int64_t R = VARLEN ? p.total : p.N;
+        const int64_t r = static_cast<int64_t>(VARLEN ? tok0 : 0) + q;
+        float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
+        // 64 columns at a time; the tile's columns are released once the last
+        // load has landed (the atomics then run from registers)
 #pragma unroll 1
-      for (int cg = 0; cg < D / 32; cg += 2) {
-        uint32_t a[2][32];
-        tmem_ld32(lane_base + C::TM_DQ + 32 * cg, a[0]);
-        tmem_ld32(lane_base + C::TM_DQ + 32 * (cg + 1), a[1]);
-        tmem_wait_ld(a[0]);
-        tmem_wait_ld(a[1]);
-        if (cg + 2 >= D / 32) {
-          tc_fence_before();
-          mbar_arrive(bar(C::BAR_DQ_EMPTY));
-        }
-        if (q < L) {
+        for (int cg = 0; cg < D / 32; cg += 2) {
+          uint32_t a[2][32];
+          tmem_ld32(lane_base + C::TM_DQ + 32 * cg, a[0]);
+          tmem_ld32(lane_base + C::TM_DQ + 32 * (cg + 1), a[1]);
+          tmem_wait_ld(a[0]);
+          tmem_wait_ld(a[1]);
+          if (cg + 2 >= D / 32) {
+            tc_fence_before();
+            mbar_arrive(bar(C::BAR_DQ_EMPTY));
+          }
+          if (q < L) {
 #pragma unroll
-          for (int e = 0; e < 2; ++e)
+            for (int e = 0; e < 2; ++e)
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
-              atomicAdd(acc4 + dq_acc_index4(bh_, 8 * (cg + e) + u, r, R, D),
-                        make_float4(__uint_as_float(a[e][4 * u]), __uint_as_float(a[e][4 * u + 1]),
-                                    __uint_as_float(a[e][4 * u + 2]), __uint_as_float(a[e][4 * u + 3])));
+              for (int u = 0; u < 8; ++u)
+                atomicAdd(acc4 + dq_acc_index4(bh_, 8 * (cg + e) + u, r, R, D),
+                          make_float4(__uint_as_float(a[e][4 * u]), __uint_as_float(a[e][4 * u + 1]),
+                                      __uint_as_float(a[e][4 * u + 2]), __uint_as_float(a[e][4 * u + 3])));
+          }
         }
       }
     }

@@ -101,6 +101,27 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
                         const int* cu_seqlens, int nseq, int total, int max_seqlen,
                         int H, int d, float scale, int causal, void* stream);
 
+/* Deterministic backward, dense batch ("FlashAttention-2 (PT)", section
+ * "Desempenho e eficiencia": the method is exact and deterministic).
+ * Arguments, layouts, workspace size and errors are those of fa_bwd.  The
+ * outputs are bitwise reproducible from run to run: dK and dV come from the
+ * same fused pass (without its dQ product), and dQ from a second pass in
+ * which one CTA per 128-row query tile sums the key tiles in increasing
+ * order in tensor memory (S and dP are recomputed there; no atomics).  Only
+ * the D part of the workspace is used.  About 1.4x the matrix work of
+ * fa_bwd. */
+fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
+                               const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
+                               int B, int N, int H, int d, float scale, int causal, void* stream);
+
+/* Deterministic backward, packed variable-length batch.  Arguments as
+ * fa_varlen_bwd; results bitwise reproducible as for fa_bwd_deterministic. */
+fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* v, const void* o,
+                                      const float* lse, const void* dO, void* dq, void* dk, void* dv,
+                                      void* workspace, size_t ws_bytes, const int* cu_seqlens, int nseq,
+                                      int total, int max_seqlen, int H, int d, float scale, int causal,
+                                      void* stream);
+
 /* Backward pass, dense batch, for callers that cannot allocate device memory.
  * There is no counterpart to this in the method's description: it exists for
  * callers that may not call cudaMalloc (or any allocating routine) when they

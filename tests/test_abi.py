@@ -62,6 +62,12 @@ def test_host_validation(L):
     assert L.fa_bwd(*args, ws - 1, 1, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_WORKSPACE
     assert L.fa_bwd(*args[:9], P + 16, ws, 1, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG  # ws not 256-aligned
     assert L.fa_bwd(*args, ws, 1, 8, 1, 128, 1.0, 3, None) == fa.FA_ERR_INVALID_ARG
+    # the deterministic entry points validate exactly as fa_bwd / fa_varlen_bwd
+    assert L.fa_bwd_deterministic(*args, ws - 1, 1, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert L.fa_bwd_deterministic(*args, ws, 1, 8, 1, 96, 1.0, 0, None) == fa.FA_ERR_UNSUPPORTED
+    assert L.fa_bwd_deterministic(None, *args[1:], ws, 1, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_varlen_bwd_deterministic(*args, ws, None, 1, 8, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_varlen_bwd_deterministic(*args, ws, P + 2, 1, 8, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="host without a GPU driver only")
