@@ -41,7 +41,7 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from workloads import WORKLOADS, make_dense, make_workload  # noqa: E402
+from workloads import DECODE_WORKLOADS, WORKLOADS, make_decode, make_dense, make_workload  # noqa: E402
 
 WORKLOAD = "fwd_bwd_causal_b4_h16_n4096_d128_qk2x"
 METRIC = "attention TFLOP/s fwd+bwd (bf16), fraction of B200 dense BF16 peak"
@@ -404,8 +404,11 @@ def run_sweep(args):
     iters = max(30, args.calls)
     # a buffer larger than L2, written between calls for the flushed variant
     flush_buf = torch.empty(256 << 20, dtype=torch.uint8, device=dev)
-    names = [args.only] if args.only else list(WORKLOADS)
+    names = [args.only] if args.only else list(WORKLOADS) + list(DECODE_WORKLOADS)
     for name in names:
+        if name in DECODE_WORKLOADS:
+            _sweep_decode(fa, DECODE_WORKLOADS[name], args, dev, stream, peaks, iters)
+            continue
         w = WORKLOADS[name]
         x = {k: (v.to(dev) if isinstance(v, torch.Tensor) else v) for k, v in make_workload(w, seed=args.seed).items()}
         scale = 1.0 / math.sqrt(w.d)
@@ -479,6 +482,46 @@ def run_sweep(args):
                                  "datasheet_2250": tf / DATASHEET_BF16_TFLOPS, "peak_source": peaks["source"]},
                         "clocks": clk}), flush=True)
         del x
+
+
+def _sweep_decode(fa, w, args, dev, stream, peaks, iters):
+    """Decode lines: HBM-bound, reported as GB/s of the bytes the call must
+    move (the valid K and V cache rows, q, o and lse) against the measured
+    copy bandwidth."""
+    x = {k: v.to(dev) for k, v in make_decode(w.B, w.Nq, w.Nk, w.H, w.d, w.lo, w.hi, seed=args.seed).items()}
+    lens = x["seqlens"].tolist()
+    o = torch.empty_like(x["q"])
+    lse = torch.empty((w.B, w.H, w.Nq), dtype=torch.float32, device=dev)
+    nws = fa.decode_workspace_size(w.B, w.Nq, w.Nk, w.H, w.d)
+    ws = torch.empty(max(nws, 256), dtype=torch.uint8, device=dev)
+    nbytes = sum(lens) * w.H * w.d * 2 * 2 + 2 * w.B * w.Nq * w.H * w.d * 2 + w.B * w.H * w.Nq * 4
+
+    def fn():
+        fa.decode_fwd(x["q"], x["k"], x["v"], x["seqlens"], causal=True, out=o, lse=lse, workspace=ws)
+    for _ in range(10):
+        fn()
+    fa.check_device_error()
+    evs = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(iters)]
+    clocks = ClockSampler(0)
+    torch.cuda.synchronize(dev)
+    clocks.start()
+    for e0, e1 in evs:
+        e0.record(stream)
+        fn()
+        e1.record(stream)
+    torch.cuda.synchronize(dev)
+    clk = clocks.stop()
+    fa.check_device_error()
+    ms = [e0.elapsed_time(e1) for e0, e1 in evs]
+    med = statistics.median(ms)
+    gbs = nbytes / (med * 1e-3) / 1e9
+    print(json.dumps({
+        "sweep": w.name, "causal": True, "direction": "decode_fwd", "calls": iters, "warmup": 10,
+        "l2": f"cache ({nbytes / 2**30:.2f} GiB) larger than the 126 MB L2; not flushed",
+        "shape": {"B": w.B, "Nq": w.Nq, "Nk": w.Nk, "H": w.H, "d": w.d, "seqlens_sum": sum(lens)},
+        "bytes": nbytes, "ms": {"min": min(ms), "median": med, "p90": _pct(ms, 0.9)},
+        "gbs_at_median": gbs, "frac": {"measured_hbm": gbs / peaks["hbm_gbs"], "peak_source": peaks["source"]},
+        "clocks": clk}), flush=True)
 
 
 def main():

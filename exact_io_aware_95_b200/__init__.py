@@ -19,6 +19,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FaError", "lib", "fwd", "bwd", "varlen_fwd", "varlen_bwd", "workspace_size", "check_device_error",
+           "decode_fwd", "decode_workspace_size",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FA_ERR_WORKSPACE",
            "EXPORTS", "LIB_PATH"]
 
@@ -41,6 +42,8 @@ EXPORTS = {
     "fa_bwd_deterministic": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
     "fa_varlen_bwd_deterministic": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _I, _I, _I, _I, _I, _F, _I,
                                          _P]),
+    "fa_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "fa_decode_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_P]),
@@ -208,6 +211,44 @@ def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, c
                 _stream_ptr(q))
     _check(st, "fa_varlen_bwd_deterministic" if deterministic else "fa_varlen_bwd")
     return dq, dk, dv
+
+
+def decode_workspace_size(B: int, Nq: int, Nk: int, H: int, d: int) -> int:
+    return int(lib().fa_decode_workspace_size(B, Nq, Nk, H, d))
+
+
+def decode_fwd(q, k_cache, v_cache, seqlens_k: Optional[torch.Tensor] = None, causal: bool = False,
+               scale: Optional[float] = None, out=None, lse=None, workspace=None):
+    """Decode-shaped forward: q [B, Nq, H, d] (Nq <= 16) against caches
+    [B, Nk, H, d] with seqlens_k int32 [B] valid rows per entry (None: all).
+    Returns O [B, Nq, H, d] bf16 and LSE [B, H, Nq] fp32."""
+    _need(q, "q", torch.bfloat16, 4)
+    _need(k_cache, "k_cache", torch.bfloat16, 4)
+    _need(v_cache, "v_cache", torch.bfloat16, 4)
+    B, Nq, H, d = q.shape
+    Nk = k_cache.shape[1]
+    if k_cache.shape != (B, Nk, H, d) or v_cache.shape != k_cache.shape:
+        raise ValueError("k_cache and v_cache must be [B, Nk, H, d] matching q")
+    if seqlens_k is not None:
+        _need(seqlens_k, "seqlens_k", torch.int32, 1)
+        if seqlens_k.numel() != B:
+            raise ValueError("seqlens_k must have B entries")
+    o = torch.empty_like(q) if out is None else out
+    l = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws_need = decode_workspace_size(B, Nq, Nk, H, d)
+    ws = workspace
+    if ws is None and ws_need > 0:
+        ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    ts = [q, k_cache, v_cache, o, l] + [t for t in (seqlens_k, ws) if t is not None]
+    _same_device(*ts)
+    with _on(q):
+        st = lib().fa_decode_fwd(q.data_ptr(), k_cache.data_ptr(), v_cache.data_ptr(), o.data_ptr(), l.data_ptr(),
+                                 None if seqlens_k is None else seqlens_k.data_ptr(),
+                                 None if ws is None else ws.data_ptr(),
+                                 0 if ws is None else ws.numel() * ws.element_size(),
+                                 B, Nq, Nk, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
+    _check(st, "fa_decode_fwd")
+    return o, l
 
 
 def check_device_error(stream: Optional[torch.cuda.Stream] = None):

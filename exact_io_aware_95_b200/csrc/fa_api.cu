@@ -16,6 +16,7 @@
 #endif
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
+#include "fa_decode.cuh"
 #include "fa_fwd.cuh"
 
 namespace {
@@ -364,6 +365,62 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
                  : dispatch_bwd<128>(dev, causal, varlen, mq, mk, mv, mdo, p, dq_group, det, s);
 }
 
+// ----------------------------------------------------------------- decode
+// Key ranges per (batch entry, head): about FA_DECODE_TARGET_WAVES waves of
+// two CTAs per SM on a 148-SM part, so the block scheduler can even out
+// ranges of unequal work (ragged cache lengths), with at least
+// FA_DECODE_MIN_TILES 64-key tiles per range.
+// The choice depends on the sizes only, so the workspace size is a function
+// of the sizes.
+#ifndef FA_DECODE_TARGET_WAVES
+#define FA_DECODE_TARGET_WAVES 8
+#endif
+#ifndef FA_DECODE_MIN_TILES
+#define FA_DECODE_MIN_TILES 4
+#endif
+constexpr int64_t kDecodeTargetCtas = int64_t(FA_DECODE_TARGET_WAVES) * 2 * 148;
+constexpr int kDecodeTileKeys = 64;
+
+void decode_split(int B, int H, int Nk, int* nsplit, int* tiles_per_split) {
+  const int ntiles = Nk > 0 ? (Nk + kDecodeTileKeys - 1) / kDecodeTileKeys : 1;
+  const int64_t pairs = static_cast<int64_t>(B) * H;
+  int64_t ns = (kDecodeTargetCtas + pairs - 1) / pairs;
+  if (ns > ntiles / FA_DECODE_MIN_TILES) ns = ntiles / FA_DECODE_MIN_TILES;
+  if (ns > fa::kDecodeMaxSplits) ns = fa::kDecodeMaxSplits;
+  if (ns < 1) ns = 1;
+  const int tps = static_cast<int>((ntiles + ns - 1) / ns);
+  *tiles_per_split = tps;
+  *nsplit = (ntiles + tps - 1) / tps;
+}
+
+size_t decode_ws_bytes(int B, int Nq, int Nk, int H, int d) {
+  int ns, tps;
+  decode_split(B, H, Nk, &ns, &tps);
+  if (ns == 1) return 0;
+  const size_t rows = static_cast<size_t>(B) * H * ns * Nq;
+  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+}
+
+template <int D, int NQ>
+fa_status launch_decode(int dev, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
+                        cudaStream_t s) {
+  static bool done[kMaxDevices] = {};
+  auto kern = fa::fa_decode_split_kernel<D, NQ>;
+  constexpr int smem = fa::DecCfg<D, NQ>::SMEM_BYTES;
+  static_assert(fa::DecCfg<D, NQ>::KT == kDecodeTileKeys, "tile size of the split choice");
+  fa_status st = ensure_smem(kern, dev, smem, done);
+  if (st != FA_OK) return st;
+  kern<<<dim3(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.H), static_cast<unsigned>(p.B)),
+         fa::DecCfg<D, NQ>::THREADS, smem, s>>>(mk, mv, p);
+  if ((st = launch_status()) != FA_OK) return st;
+  if (p.nsplit > 1) {
+    const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Nq;
+    fa::fa_decode_merge_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, s>>>(p);
+    if ((st = launch_status()) != FA_OK) return st;
+  }
+  return FA_OK;
+}
+
 bool valid_cu(const int* cu, int nseq, int total, int max_seqlen) {
   return cu && nseq >= 1 && total >= 1 && max_seqlen >= 1;
 }
@@ -422,6 +479,55 @@ fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* 
                     scale, causal, stream, true);
 }
 
+size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d) {
+  if (B < 1 || Nq < 1 || Nq > 16 || Nk < 1 || H < 1 || (d != 64 && d != 128)) return 0;
+  return decode_ws_bytes(B, Nq, Nk, H, d);
+}
+
+fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                        const int* seqlens_k, void* workspace, size_t ws_bytes, int B, int Nq, int Nk, int H, int d,
+                        float scale, int causal, void* stream) {
+  if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
+    return FA_ERR_INVALID_ARG;
+  if (seqlens_k && (reinterpret_cast<uintptr_t>(seqlens_k) & 3u) != 0) return FA_ERR_INVALID_ARG;
+  if (B < 1 || Nq < 1 || Nk < 1 || H < 1) return FA_ERR_INVALID_ARG;
+  if (Nq > 16) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;  // grid y / z limits
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
+  if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
+  if (static_cast<int64_t>(B) * Nk * H * d > (int64_t(1) << 40)) return FA_ERR_INVALID_ARG;
+  const size_t need = decode_ws_bytes(B, Nq, Nk, H, d);
+  if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
+  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  int dev;
+  fa_status st = current_device(&dev);
+  if (st != FA_OK) return st;
+  CUtensorMap mk, mv;
+  if ((st = make_map_bf16(&mk, k_cache, d, H, Nk, B, kDecodeTileKeys)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mv, v_cache, d, H, Nk, B, kDecodeTileKeys)) != FA_OK) return st;
+  fa::DecParams p;
+  p.q = q;
+  p.o = o;
+  p.lse = lse;
+  p.seqlens = seqlens_k;
+  p.B = B;
+  p.Nq = Nq;
+  p.Nk = Nk;
+  p.H = H;
+  decode_split(B, H, Nk, &p.nsplit, &p.tiles_per_split);
+  const size_t rows = static_cast<size_t>(B) * H * p.nsplit * Nq;
+  p.part_o = p.nsplit > 1 ? static_cast<float*>(workspace) : nullptr;
+  p.part_lse = p.nsplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * d * sizeof(float)))
+                            : nullptr;
+  p.causal = causal;
+  p.scale_log2 = scale * kLog2e;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  if (d == 64) return Nq == 1 ? launch_decode<64, 1>(dev, mk, mv, p, s) : launch_decode<64, 16>(dev, mk, mv, p, s);
+  return Nq == 1 ? launch_decode<128, 1>(dev, mk, mv, p, s) : launch_decode<128, 16>(dev, mk, mv, p, s);
+}
+
 const char* fa_status_string(fa_status s) {
   switch (s) {
     case FA_OK: return "ok";
@@ -446,7 +552,8 @@ fa_status fa_get_device_error(void* stream) {
     cudaGetLastError();
     return FA_ERR_CUDA;
   }
-  return word ? FA_ERR_TIMEOUT : FA_OK;
+  if (word & fa::FA_DEVERR_TIMEOUT) return FA_ERR_TIMEOUT;
+  return word ? FA_ERR_INVALID_ARG : FA_OK;
 }
 
 }  // extern "C"

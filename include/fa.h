@@ -122,6 +122,32 @@ fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* 
                                       int total, int max_seqlen, int H, int d, float scale, int causal,
                                       void* stream);
 
+/* Bytes of workspace fa_decode_fwd needs for these sizes (fp32 partial
+ * outputs and logsumexps of the key ranges, 256-byte aligned).  0 when the
+ * sizes need none (one key range covers the cache) or are invalid. */
+size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d);
+
+/* Decode-shaped forward: Nq new queries per batch entry (1 <= Nq <= 16)
+ * against a cache of up to Nk keys and values.  The method's tiling and
+ * online softmax ("FlashAttention: Fast and Memory-Efficient Exact
+ * Attention with IO-Awareness", sections "Tiling" and "Softmax en linea")
+ * applied over ranges of the cache in parallel, the ranges merged exactly
+ * through their logsumexps.
+ * q, o: bf16 [B, Nq, H, d]; k_cache, v_cache: bf16 [B, Nk, H, d];
+ * lse: fp32 [B, H, Nq] output (natural log).
+ * seqlens_k: int32 device array [B] of valid cache rows per batch entry
+ * (0 <= L_b <= Nk), or NULL for all Nk; rows past L_b are never used in the
+ * arithmetic (they may hold anything).  A value outside [0, Nk] is reported
+ * by fa_get_device_error() and that entry's outputs are not written.
+ * causal = 1: query i is the token at position L_b - Nq + i and sees keys
+ * j <= L_b - Nq + i; a query that sees no key gets O = 0 and LSE = -inf.
+ * workspace: device buffer of ws_bytes >= fa_decode_workspace_size(...),
+ * 256-byte aligned (may be NULL when that size is 0).
+ * Returns FA_ERR_UNSUPPORTED for Nq > 16 or d not in {64, 128}. */
+fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
+                        const int* seqlens_k, void* workspace, size_t ws_bytes,
+                        int B, int Nq, int Nk, int H, int d, float scale, int causal, void* stream);
+
 /* Backward pass, dense batch, for callers that cannot allocate device memory.
  * There is no counterpart to this in the method's description: it exists for
  * callers that may not call cudaMalloc (or any allocating routine) when they
@@ -149,8 +175,11 @@ fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void
 const char* fa_status_string(fa_status s);
 
 /* Synchronises `stream`, then reads and clears this device's error word.
- * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call,
- * FA_ERR_CUDA if the synchronisation itself failed, else FA_OK. */
+ * FA_ERR_TIMEOUT if a kernel gave up on a bounded wait since the last call;
+ * otherwise FA_ERR_INVALID_ARG if a kernel found device-side sizes that
+ * contradict the call (cu_seqlens offsets past `total` or longer than
+ * max_seqlen, seqlens_k outside [0, Nk]) and skipped that work;
+ * FA_ERR_CUDA if the synchronisation itself failed; else FA_OK. */
 fa_status fa_get_device_error(void* stream);
 
 #ifdef __cplusplus

@@ -26,7 +26,8 @@ from typing import Dict, List, Optional
 
 import torch
 
-__all__ = ["Workload", "WORKLOADS", "make_dense", "make_varlen", "varlen_lengths", "cu_seqlens_of"]
+__all__ = ["Workload", "WORKLOADS", "make_dense", "make_varlen", "varlen_lengths", "cu_seqlens_of",
+           "DecodeWorkload", "DECODE_WORKLOADS", "make_decode"]
 
 
 @dataclass(frozen=True)
@@ -115,3 +116,40 @@ def make_workload(w: Workload, seed: int = 0) -> Dict[str, torch.Tensor]:
         lens = varlen_lengths(w.varlen_total, w.varlen_lo, w.varlen_hi, seed)
         return make_varlen(lens, w.H, w.d, seed, with_grad=w.backward)
     return make_dense(w.B, w.N, w.H, w.d, seed, w.qk_scale_factor, with_grad=True)
+
+
+@dataclass(frozen=True)
+class DecodeWorkload:
+    """Decode-shaped inputs: Nq new queries per batch entry against a cache of
+    Nk rows, of which seqlens are valid (all Nk when lo == hi == Nk)."""
+    name: str
+    B: int
+    Nq: int
+    Nk: int
+    H: int
+    d: int
+    lo: int
+    hi: int
+
+
+# Serving-style decode: one new token per sequence against a 16k-token cache,
+# with every cache full, and with lengths spread over [1024, 16384].
+DECODE_WORKLOADS: Dict[str, DecodeWorkload] = {
+    "decode_b16_h16_nk16384_d128_full": DecodeWorkload("decode_b16_h16_nk16384_d128_full", 16, 1, 16384, 16, 128,
+                                                       16384, 16384),
+    "decode_b16_h16_nk16384_d128_ragged": DecodeWorkload("decode_b16_h16_nk16384_d128_ragged", 16, 1, 16384, 16,
+                                                         128, 1024, 16384),
+}
+
+
+def make_decode(B: int, Nq: int, Nk: int, H: int, d: int, lo: int, hi: int, seed: int = 0) -> Dict[str, torch.Tensor]:
+    """q [B, Nq, H, d], k, v caches [B, Nk, H, d] (bf16, fp32 randn drawn in
+    the order q, k, v from one generator), and seqlens int32 [B] drawn
+    uniformly from [lo, hi] by a second generator seeded with ``seed``."""
+    gen = torch.Generator(device="cpu").manual_seed(seed)
+    q = torch.randn((B, Nq, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    k = torch.randn((B, Nk, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    v = torch.randn((B, Nk, H, d), generator=gen, dtype=torch.float32).to(torch.bfloat16)
+    g2 = torch.Generator(device="cpu").manual_seed(seed)
+    lens = torch.randint(lo, hi + 1, (B,), generator=g2, dtype=torch.int64).to(torch.int32)
+    return {"q": q, "k": k, "v": v, "seqlens": lens}
