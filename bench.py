@@ -41,7 +41,8 @@ sys.path.insert(0, ROOT)
 
 import torch  # noqa: E402
 
-from workloads import DECODE_WORKLOADS, WORKLOADS, make_decode, make_dense, make_workload  # noqa: E402
+from workloads import (DECODE_WORKLOADS, WORKLOADS, make_decode, make_dense, make_fp8_dense,  # noqa: E402
+                       make_workload)
 
 WORKLOAD = "fwd_bwd_causal_b4_h16_n4096_d128_qk2x"
 METRIC = "attention TFLOP/s fwd+bwd (bf16), fraction of B200 dense BF16 peak"
@@ -449,6 +450,16 @@ def run_sweep(args):
             # FLOPs (2.5x forward); its recomputation of S and dP is not counted
             dirs = [("fwd", f, ff)] + ([("bwd", b, 2.5 * ff), ("bwd_deterministic", lambda: b(True), 2.5 * ff)]
                                        if w.backward else [])
+            if not w.varlen_total and w.d == 128:
+                # the 8-bit forward on the same draws, quantized per tensor
+                x8, sc = make_fp8_dense(w.B, w.N, w.H, w.d, seed=args.seed, qk_scale_factor=w.qk_scale_factor)
+                x8 = {n: t.to(dev) for n, t in x8.items()}
+                ws8 = torch.empty(fa.fwd_fp8_workspace_size(w.B, w.N, w.H, w.d), dtype=torch.uint8, device=dev)
+
+                def f8():
+                    fa.fwd_fp8(x8["q"], x8["k"], x8["v"], sc["q"], sc["k"], sc["v"], causal=causal, scale=scale,
+                               out=o, lse=lse, workspace=ws8)
+                dirs.append(("fwd_fp8", f8, ff))
             for direction, fn, flops in dirs:
                 for flush in flush_variants:
                     for _ in range(10):

@@ -19,7 +19,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FaError", "lib", "fwd", "bwd", "varlen_fwd", "varlen_bwd", "workspace_size", "check_device_error",
-           "decode_fwd", "decode_workspace_size",
+           "decode_fwd", "decode_workspace_size", "fwd_fp8", "fwd_fp8_workspace_size",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FA_ERR_WORKSPACE",
            "EXPORTS", "LIB_PATH"]
 
@@ -43,6 +43,8 @@ EXPORTS = {
     "fa_varlen_bwd_deterministic": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _P, _S, _P, _I, _I, _I, _I, _I, _F, _I,
                                          _P]),
     "fa_decode_workspace_size": (_S, [_I, _I, _I, _I, _I]),
+    "fa_fwd_fp8_workspace_size": (_S, [_I, _I, _I, _I]),
+    "fa_fwd_fp8": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
@@ -211,6 +213,35 @@ def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, c
                 _stream_ptr(q))
     _check(st, "fa_varlen_bwd_deterministic" if deterministic else "fa_varlen_bwd")
     return dq, dk, dv
+
+
+def fwd_fp8_workspace_size(B: int, N: int, H: int, d: int) -> int:
+    return int(lib().fa_fwd_fp8_workspace_size(B, N, H, d))
+
+
+def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causal: bool = False,
+            scale: Optional[float] = None, out=None, lse=None, workspace=None):
+    """Forward with e4m3 inputs [B, N, H, 128] (torch.float8_e4m3fn): attention of
+    descale_q*q, descale_k*k, descale_v*v.  Returns O bf16 [B, N, H, 128], LSE [B, H, N]."""
+    for t, n in ((q, "q"), (k, "k"), (v, "v")):
+        _need(t, n, torch.float8_e4m3fn, 4)
+    if k.shape != q.shape or v.shape != q.shape:
+        raise ValueError("q, k, v must have the same shape [B, N, H, d]")
+    B, N, H, d = q.shape
+    o = torch.empty(q.shape, dtype=torch.bfloat16, device=q.device) if out is None else out
+    l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
+    ws = workspace
+    if ws is None:
+        ws = torch.empty(max(fwd_fp8_workspace_size(B, N, H, d), 256), dtype=torch.uint8, device=q.device)
+    _need(o, "out", torch.bfloat16, 4)
+    _same_device(q, k, v, o, l, ws)
+    with _on(q):
+        st = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(descale_q), float(descale_k),
+                              float(descale_v), o.data_ptr(), l.data_ptr(), ws.data_ptr(),
+                              ws.numel() * ws.element_size(), B, N, H, d, _scale(scale, d), int(bool(causal)),
+                              _stream_ptr(q))
+    _check(st, "fa_fwd_fp8")
+    return o, l
 
 
 def decode_workspace_size(B: int, Nq: int, Nk: int, H: int, d: int) -> int:

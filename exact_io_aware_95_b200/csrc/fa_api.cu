@@ -18,6 +18,7 @@
 #include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
 #include "fa_fwd.cuh"
+#include "fa_fwd_fp8.cuh"
 
 namespace {
 
@@ -145,6 +146,23 @@ fa_status make_map_bf16(CUtensorMap* m, const void* base, int d, int H, int64_t 
   cuuint32_t box[4] = {64, 1, (cuuint32_t)box_rows, 1};
   cuuint32_t estr[4] = {1, 1, 1, 1};
   CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_BFLOAT16, 4, const_cast<void*>(base), dims, strides, box, estr,
+                   CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                   CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
+}
+
+// Tensor map over a byte array (e4m3) with dims {d0, d1, d2, d3} (d0
+// innermost, contiguous), row pitches in bytes, boxes {b0, b1, b2, 1} and
+// 128-byte swizzle.
+fa_status make_map_u8(CUtensorMap* m, const void* base, const uint64_t (&dims)[4], const uint64_t (&pitch)[3],
+                      const uint32_t (&box)[3]) {
+  EncodeTiledFn enc = encode_fn();
+  if (!enc) return FA_ERR_CUDA;
+  cuuint64_t gd[4] = {dims[0], dims[1], dims[2], dims[3]};
+  cuuint64_t gs[3] = {pitch[0], pitch[1], pitch[2]};
+  cuuint32_t bx[4] = {box[0], box[1], box[2], 1};
+  cuuint32_t estr[4] = {1, 1, 1, 1};
+  CUresult r = enc(m, CU_TENSOR_MAP_DATA_TYPE_UINT8, 4, const_cast<void*>(base), gd, gs, bx, estr,
                    CU_TENSOR_MAP_INTERLEAVE_NONE, CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
                    CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
@@ -526,6 +544,71 @@ fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
   if (d == 64) return Nq == 1 ? launch_decode<64, 1>(dev, mk, mv, p, s) : launch_decode<64, 16>(dev, mk, mv, p, s);
   return Nq == 1 ? launch_decode<128, 1>(dev, mk, mv, p, s) : launch_decode<128, 16>(dev, mk, mv, p, s);
+}
+
+size_t fa_fwd_fp8_workspace_size(int B, int N, int H, int d) {
+  if (B < 1 || N < 1 || H < 1 || d != 128) return 0;
+  const size_t npad = (static_cast<size_t>(N) + 15) / 16 * 16;
+  return align256(static_cast<size_t>(B) * H * 128 * npad);
+}
+
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
+                     void* o, float* lse, void* workspace, size_t ws_bytes, int B, int N, int H, int d, float scale,
+                     int causal, void* stream) {
+  if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
+  if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  if (B < 1 || N < 1 || H < 1) return FA_ERR_INVALID_ARG;
+  if (causal != 0 && causal != 1) return FA_ERR_INVALID_ARG;
+  if (!std::isfinite(scale) || !std::isfinite(descale_q) || !std::isfinite(descale_k) || !std::isfinite(descale_v) ||
+      !(descale_q > 0.f) || !(descale_k > 0.f) || !(descale_v > 0.f))
+    return FA_ERR_INVALID_ARG;
+  if (d != 128) return FA_ERR_UNSUPPORTED;
+  if (B > 65535 || H > 65535) return FA_ERR_INVALID_ARG;  // transpose grid y / z
+  if (static_cast<int64_t>(B) * N * H * d > (int64_t(1) << 40)) return FA_ERR_INVALID_ARG;
+  if (ws_bytes < fa_fwd_fp8_workspace_size(B, N, H, d)) return FA_ERR_WORKSPACE;
+  int dev;
+  fa_status st = current_device(&dev);
+  if (st != FA_OK) return st;
+  const uint64_t npad = (static_cast<uint64_t>(N) + 15) / 16 * 16;
+  CUtensorMap mq, mk, mvt;
+  {
+    const uint64_t dims[4] = {128, static_cast<uint64_t>(H), static_cast<uint64_t>(N), static_cast<uint64_t>(B)};
+    const uint64_t pitch[3] = {128, static_cast<uint64_t>(H) * 128, static_cast<uint64_t>(N) * H * 128};
+    const uint32_t box[3] = {128, 1, 128};
+    if ((st = make_map_u8(&mq, q, dims, pitch, box)) != FA_OK) return st;
+    if ((st = make_map_u8(&mk, k, dims, pitch, box)) != FA_OK) return st;
+  }
+  {
+    const uint64_t dims[4] = {npad, 128, static_cast<uint64_t>(H), static_cast<uint64_t>(B)};
+    const uint64_t pitch[3] = {npad, 128 * npad, static_cast<uint64_t>(H) * 128 * npad};
+    const uint32_t box[3] = {128, 128, 1};
+    if ((st = make_map_u8(&mvt, workspace, dims, pitch, box)) != FA_OK) return st;
+  }
+  static bool done_nc[kMaxDevices] = {}, done_c[kMaxDevices] = {};
+  auto kern = causal ? fa::fa_fwd_fp8_kernel<true> : fa::fa_fwd_fp8_kernel<false>;
+  constexpr int smem = fa::Fp8Cfg::SMEM_BYTES;
+  if ((st = ensure_smem(kern, dev, smem, causal ? done_c : done_nc, fa::kLaunchRegs)) != FA_OK) return st;
+  cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  fa::fa_fp8_transpose_v_kernel<<<dim3(static_cast<unsigned>((npad + 127) / 128), static_cast<unsigned>(H),
+                                       static_cast<unsigned>(B)),
+                                  128, 0, s>>>(static_cast<const uint8_t*>(v), static_cast<uint8_t*>(workspace), N,
+                                               H, static_cast<int>(npad));
+  if ((st = launch_status()) != FA_OK) return st;
+  fa::Fp8Params p;
+  p.o = o;
+  p.lse = lse;
+  p.B = B;
+  p.N = N;
+  p.H = H;
+  p.npairs = (N + 255) / 256;
+  p.group = head_group(static_cast<int64_t>(N) * 128 * 2, static_cast<int64_t>(B) * H);  // K and V^T bytes
+  p.scale_log2 = scale * descale_q * descale_k * kLog2e;
+  p.descale_v = descale_v;
+  const int64_t grid = static_cast<int64_t>(p.npairs) * B * H;
+  if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
+  kern<<<static_cast<unsigned>(grid), fa::Fp8Cfg::THREADS, smem, s>>>(mq, mk, mvt, p);
+  return launch_status();
 }
 
 const char* fa_status_string(fa_status s) {

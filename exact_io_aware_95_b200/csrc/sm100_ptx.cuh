@@ -140,6 +140,17 @@ __device__ __forceinline__ void umma_ts(uint32_t d_tmem, uint32_t a_tmem, uint64
       "r"(a_tmem), "l"(bdesc), "r"(idesc), "r"(accumulate)
       : "memory");
 }
+// D[tmem] (+)= A[smem] * B[smem]^T, kind::f8f6f4 (here: e4m3 inputs, fp32
+// accumulate).  One instruction covers K = 32 (32 bytes of each operand row).
+__device__ __forceinline__ void umma_ss_f8(uint32_t d_tmem, uint64_t adesc, uint64_t bdesc, uint32_t idesc,
+                                           uint32_t accumulate) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}\n" ::"r"(d_tmem),
+      "l"(adesc), "l"(bdesc), "r"(idesc), "r"(accumulate)
+      : "memory");
+}
 // Arrive once on the mbarrier when every tcgen05 op issued so far by this
 // thread has completed.
 __device__ __forceinline__ void umma_commit(uint32_t bar) {
@@ -168,6 +179,16 @@ __device__ __forceinline__ uint64_t sdesc_sw128(uint32_t saddr, uint32_t lbo_byt
 // issuing thread far ahead of the tensor core.
 __device__ __forceinline__ uint64_t sdesc_adv(uint64_t desc, uint32_t byte_off) {
   return desc + static_cast<uint64_t>(byte_off >> 4);
+}
+
+// Instruction descriptor for kind::f8f6f4 with e4m3 A/B (format code 0),
+// both K-major, and fp32 D.
+__host__ __device__ constexpr uint32_t idesc_e4m3_f32(int M, int N) {
+  return (1u << 4)                                // D format: f32
+         | (0u << 7)                              // A format: e4m3
+         | (0u << 10)                             // B format: e4m3
+         | (static_cast<uint32_t>(N >> 3) << 17)  // N / 8
+         | (static_cast<uint32_t>(M >> 4) << 24); // M / 16
 }
 
 // Instruction descriptor for kind::f16 with bf16 A/B and fp32 D.

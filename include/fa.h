@@ -122,6 +122,26 @@ fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* 
                                       int total, int max_seqlen, int H, int d, float scale, int causal,
                                       void* stream);
 
+/* Bytes of workspace fa_fwd_fp8 needs: V transposed to e4m3 [B, H, 128,
+ * Npad] with Npad = N rounded up to a multiple of 16, 256-byte aligned.
+ * 0 for invalid sizes (d must be 128). */
+size_t fa_fwd_fp8_workspace_size(int B, int N, int H, int d);
+
+/* Forward with 8-bit inputs ("FlashAttention-2 (PT)", section
+ * "FlashAttention-3": FP8 support).  q, k, v: e4m3 (OCP FP8, bias 7, no
+ * infinities) [B, N, H, 128]; the inputs the attention is taken of are
+ * descale_q * q, descale_k * k and descale_v * v (each descale finite and
+ * > 0).  o: bf16 [B, N, H, 128]; lse: fp32 [B, H, N] (natural log) of those
+ * scaled inputs.  Scores are exact products accumulated in fp32; P is
+ * rounded to e4m3 for the P V product (relative error <= 2^-4 per entry
+ * above 2^-6, absolute <= 2^-10 below) while the row sums use the unrounded
+ * P.  workspace: device buffer of ws_bytes >= fa_fwd_fp8_workspace_size(),
+ * 256-byte aligned (holds V^T for the call).  Dense batches only; d must be
+ * 128 (FA_ERR_UNSUPPORTED otherwise). */
+fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k,
+                     float descale_v, void* o, float* lse, void* workspace, size_t ws_bytes,
+                     int B, int N, int H, int d, float scale, int causal, void* stream);
+
 /* Bytes of workspace fa_decode_fwd needs for these sizes (fp32 partial
  * outputs and logsumexps of the key ranges, 256-byte aligned).  0 when the
  * sizes need none (one key range covers the cache) or are invalid. */

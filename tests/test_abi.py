@@ -15,7 +15,7 @@ ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
 def header_functions():
     txt = open(os.path.join(ROOT, "include", "fa.h")).read()
     txt = re.sub(r"/\*.*?\*/", "", txt, flags=re.S)
-    return sorted(set(re.findall(r"\b(fa_[a-z_]+)\s*\(", txt)))
+    return sorted(set(re.findall(r"\b(fa_[a-z0-9_]+)\s*\(", txt)))
 
 
 @pytest.fixture(scope="module")

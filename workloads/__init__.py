@@ -22,12 +22,12 @@ Shapes follow the pages' workloads: GPT-style training at 2k-16k context
 from __future__ import annotations
 
 from dataclasses import dataclass, field
-from typing import Dict, List, Optional
+from typing import Dict, List, Tuple, Optional
 
 import torch
 
 __all__ = ["Workload", "WORKLOADS", "make_dense", "make_varlen", "varlen_lengths", "cu_seqlens_of",
-           "DecodeWorkload", "DECODE_WORKLOADS", "make_decode"]
+           "DecodeWorkload", "DECODE_WORKLOADS", "make_decode", "quantize_e4m3", "make_fp8_dense"]
 
 
 @dataclass(frozen=True)
@@ -153,3 +153,22 @@ def make_decode(B: int, Nq: int, Nk: int, H: int, d: int, lo: int, hi: int, seed
     g2 = torch.Generator(device="cpu").manual_seed(seed)
     lens = torch.randint(lo, hi + 1, (B,), generator=g2, dtype=torch.int64).to(torch.int32)
     return {"q": q, "k": k, "v": v, "seqlens": lens}
+
+
+def quantize_e4m3(x: torch.Tensor) -> Tuple[torch.Tensor, float]:
+    """Per-tensor 8-bit input: scale = amax / 448 (the largest finite e4m3
+    value) in fp32, and x / scale converted to torch.float8_e4m3fn (round to
+    nearest even).  The attention is then taken of scale * result."""
+    amax = float(x.float().abs().max())
+    scale = amax / 448.0 if amax > 0 else 1.0
+    return (x.float() / scale).to(torch.float8_e4m3fn), scale
+
+
+def make_fp8_dense(B: int, N: int, H: int, d: int, seed: int = 0, qk_scale_factor: float = 1.0):
+    """The dense recipe (make_dense, same draws) quantized per tensor to e4m3:
+    returns {"q", "k", "v"} e4m3 tensors and {"q", "k", "v"} scales."""
+    x = make_dense(B, N, H, d, seed=seed, qk_scale_factor=qk_scale_factor, with_grad=False)
+    out, scales = {}, {}
+    for n in ("q", "k", "v"):
+        out[n], scales[n] = quantize_e4m3(x[n])
+    return out, scales
