@@ -192,7 +192,11 @@ struct BwdCfg {
   static constexpr int TM_DQ = DQ_ALIASES_DP ? TM_DP : 256 + 2 * D;
   static constexpr int TMEM_COLS = 512;
   static constexpr int THREADS = 512;
-  static constexpr int LAUNCH_REGS = 128;  // 65536 / 512; the setmaxnreg split below sums to 4 x 128
+  static constexpr int LAUNCH_REGS = 128;  // 65536 / 512
+  // setmaxnreg split per warpgroup: P/dS (two warpgroups), dQ drain,
+  // producer/MMA.  The shares add up to the launch allocation exactly.
+  static constexpr int REGS_PDS = 152, REGS_DRAIN = 104, REGS_PRODUCER = 104;
+  static_assert(2 * REGS_PDS + REGS_DRAIN + REGS_PRODUCER == 4 * LAUNCH_REGS, "register split");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
 
@@ -273,7 +277,7 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 12) {
-    regs_dec<104>();
+    regs_dec<C::REGS_PRODUCER>();
   }
   if (warp == 12) {
     // ------------------------------------------------------------ producer
@@ -337,19 +341,31 @@ __global__ void __launch_bounds__(512, 1)
         }
         umma_commit(bar(C::BAR_S));
       };
-      // Order per query tile i:  dV(i)  dP^T(i)  S^T(i+1)  dK(i)  dQ(i)
-      // so that P^T(i+1) is computed while dK(i) and dQ(i) run, and dS^T(i)
-      // while S^T(i+1) runs.
+      auto issue_dp = [&](int it) {  // dP^T = V dO_it^T
+        const uint64_t bo = dO0_k + (it % C::NSTAGE) * kStageAdv;
+#pragma unroll
+        for (int kk = 0; kk < D / 16; ++kk) {
+          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
+          umma_ss(tmem + C::TM_DP, sdesc_adv(dV_k, off), sdesc_adv(bo, off), kIdSq, kk > 0);
+        }
+        umma_commit(bar(C::BAR_DP));
+      };
+      // Order per query tile i:  dV(i)  S^T(i+1)  dK(i)  dQ(i)  dP^T(i+1).
+      // dP^T does not depend on P, so dP^T(i+1) is issued as soon as its
+      // columns are free (the P/dS warps have read dP^T(i) and, at d = 128,
+      // the drain has emptied dQ(i), which shares them): the P/dS warps then
+      // go from P^T(i+1) straight on to dS^T(i+1), and P^T(i+1) is computed
+      // while dK(i) and dQ(i) run.
       bool ok = mbar_wait(bar(C::BAR_KV), 0, abort_flag) && mbar_wait(bar(C::BAR_QDO_FULL), 0, abort_flag);
       if (ok) {
         tc_fence_after();
         issue_s(0);
+        issue_dp(0);
       }
       for (int it = 0; ok && it < niter; ++it) {
         const int st = it % C::NSTAGE;
         const uint32_t par = it & 1;
         const uint64_t q_mn = dQ0_mn + st * kStageAdv;
-        const uint64_t o_k = dO0_k + st * kStageAdv;
         const uint64_t o_mn = dO0_mn + st * kStageAdv;
         // dV += P^T dO   (A = P^T packed bf16 in tensor memory)
         if (!(ok = mbar_wait(bar(C::BAR_P), par, abort_flag))) break;
@@ -359,17 +375,6 @@ __global__ void __launch_bounds__(512, 1)
           // queries 16kk..16kk+15 of P^T: columns 8kk (first 64 queries) or 32 + 8kk (last 64)
           umma_ts(tmem + C::TM_DV, tmem + C::TM_S + kk * 8 + (kk >= 4 ? 32 : 0), sdesc_adv(o_mn, kk * 2048), kIdDV,
                   (it > 0 || kk > 0));
-        // dP^T = V dO^T  (its columns may hold the previous dQ tile: wait until drained)
-        if (DQ && C::DQ_ALIASES_DP && it > 0) {
-          if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par ^ 1u, abort_flag))) break;
-          tc_fence_after();
-        }
-#pragma unroll
-        for (int kk = 0; kk < D / 16; ++kk) {
-          const uint32_t off = (kk >> 2) * 16384 + (kk & 3) * 32;
-          umma_ss(tmem + C::TM_DP, sdesc_adv(dV_k, off), sdesc_adv(o_k, off), kIdSq, kk > 0);
-        }
-        umma_commit(bar(C::BAR_DP));
         // S^T of the next query tile (P^T(i) was consumed by dV above, in issue order)
         if (it + 1 < niter) {
           const int st1 = (it + 1) % C::NSTAGE;
@@ -396,6 +401,16 @@ __global__ void __launch_bounds__(512, 1)
         umma_commit(bar(C::BAR_QDO_EMPTY + st));
         umma_commit(bar(C::BAR_DS_EMPTY));
         if (DQ) umma_commit(bar(C::BAR_DQ_FULL));
+        // dP^T of the next query tile: the P/dS warps finished reading dP^T(i)
+        // before they signalled dS^T(i); at d = 128 its columns also hold dQ(i),
+        // so wait until the drain has loaded it (completion i of DQ_EMPTY)
+        if (it + 1 < niter) {
+          if (DQ && C::DQ_ALIASES_DP) {
+            if (!(ok = mbar_wait(bar(C::BAR_DQ_EMPTY), par, abort_flag))) break;
+            tc_fence_after();
+          }
+          issue_dp(it + 1);
+        }
       }
       if (ok) umma_commit(bar(C::BAR_ACC));
       if (*abort_flag) {
@@ -406,7 +421,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P^T and dS^T
-    regs_inc<152>();
+    regs_inc<C::REGS_PDS>();
     const int w = warp >> 2;          // this warpgroup's query columns: 64w .. 64w+63
     const int t = threadIdx.x & 127;  // key row within the tile == tensor-memory lane
     const int key = k0 + t;
@@ -548,7 +563,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ_i drain
-    regs_dec<104>();
+    regs_dec<C::REGS_DRAIN>();
     if constexpr (DQ) {
       const int t = threadIdx.x - 256;  // query row within the tile == tensor-memory lane
       const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
