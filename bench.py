@@ -156,7 +156,9 @@ def oracle_sample(w, n_heads: int, seed: int = 0):
     import numpy as np
     import oracle  # test infrastructure: only this baseline leg calls it
 
-    heads = [(0, 0), (w.B - 1, w.H - 1), (w.B // 2, w.H // 2)][:n_heads]
+    # n_heads (b, h) pairs spread evenly over the B * H heads of the workload
+    nbh = w.B * w.H
+    heads = [divmod((i * nbh) // n_heads, w.H) for i in range(n_heads)]
     key = (w.name, n_heads, seed)
     if key not in _SAMPLE_CACHE:
         x = make_dense(w.B, w.N, w.H, w.d, seed=seed, qk_scale_factor=w.qk_scale_factor)
@@ -380,7 +382,7 @@ def run_gpu(args, world, rank, local):
         "clocks": clk,
     }
     if not args.no_cpu_baseline and world == 1:
-        v, dt, desc = oracle_sample(w, 2)
+        v, dt, desc = oracle_sample(w, 16)  # about 10 s of fp64 work on the host
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc,
                                 "seconds": dt}
     return line
