@@ -137,7 +137,8 @@ size_t fa_fwd_fp8_workspace_size(int B, int N, int H, int d);
  * above 2^-6, absolute <= 2^-10 below) while the row sums use the unrounded
  * P.  workspace: device buffer of ws_bytes >= fa_fwd_fp8_workspace_size(),
  * 256-byte aligned (holds V^T for the call).  Dense batches only; d must be
- * 128 (FA_ERR_UNSUPPORTED otherwise). */
+ * 128 (FA_ERR_UNSUPPORTED otherwise); B and H at most 65535
+ * (FA_ERR_INVALID_ARG otherwise). */
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k,
                      float descale_v, void* o, float* lse, void* workspace, size_t ws_bytes,
                      int B, int N, int H, int d, float scale, int causal, void* stream);
@@ -163,7 +164,8 @@ size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d);
  * j <= L_b - Nq + i; a query that sees no key gets O = 0 and LSE = -inf.
  * workspace: device buffer of ws_bytes >= fa_decode_workspace_size(...),
  * 256-byte aligned (may be NULL when that size is 0).
- * Returns FA_ERR_UNSUPPORTED for Nq > 16 or d not in {64, 128}. */
+ * Returns FA_ERR_UNSUPPORTED for Nq > 16 or d not in {64, 128}, and
+ * FA_ERR_INVALID_ARG for B or H above 65535 (the launch grid's limits). */
 fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                         const int* seqlens_k, void* workspace, size_t ws_bytes,
                         int B, int Nq, int Nk, int H, int d, float scale, int causal, void* stream);

@@ -80,6 +80,8 @@ def test_host_validation(L):
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 1, 16384, 1, 128, 1.0, 0, None) == fa.FA_ERR_WORKSPACE
     assert L.fa_decode_fwd(P, P, P, P, P, None, P + 16, dws, 1, 1, 16384, 1, 128, 1.0, 0, None) == \
         fa.FA_ERR_INVALID_ARG  # workspace not 256-aligned
+    assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 65536, 1, 64, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 1, 64, 65536, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
 
 
 @pytest.mark.skipif(os.path.exists("/dev/nvidia0"), reason="host without a GPU driver only")
