@@ -384,59 +384,38 @@ fa_status bwd_common(const void* q, const void* k, const void* v, const void* o,
 }
 
 // ----------------------------------------------------------------- decode
-// Key ranges per (batch entry, head): about FA_DECODE_TARGET_WAVES waves of
-// two CTAs per SM on a 148-SM part, so the block scheduler can even out
-// ranges of unequal work (ragged cache lengths), with at least
-// FA_DECODE_MIN_TILES 64-key tiles per range.
-// The choice depends on the sizes only, so the workspace size is a function
-// of the sizes.
-#ifndef FA_DECODE_TARGET_WAVES
-#define FA_DECODE_TARGET_WAVES 8
-#endif
-#ifndef FA_DECODE_MIN_TILES
-#define FA_DECODE_MIN_TILES 4
-#endif
-constexpr int64_t kDecodeTargetCtas = int64_t(FA_DECODE_TARGET_WAVES) * 2 * 148;
-constexpr int kDecodeTileKeys = 64;
-
-void decode_split(int B, int H, int Nk, int* nsplit, int* tiles_per_split) {
-  const int ntiles = Nk > 0 ? (Nk + kDecodeTileKeys - 1) / kDecodeTileKeys : 1;
-  const int64_t pairs = static_cast<int64_t>(B) * H;
-  int64_t ns = (kDecodeTargetCtas + pairs - 1) / pairs;
-  if (ns > ntiles / FA_DECODE_MIN_TILES) ns = ntiles / FA_DECODE_MIN_TILES;
-  if (ns > fa::kDecodeMaxSplits) ns = fa::kDecodeMaxSplits;
-  if (ns < 1) ns = 1;
-  const int tps = static_cast<int>((ntiles + ns - 1) / ns);
-  *tiles_per_split = tps;
-  *nsplit = (ntiles + tps - 1) / tps;
-}
-
-size_t decode_ws_bytes(int B, int Nq, int Nk, int H, int d) {
-  int ns, tps;
-  decode_split(B, H, Nk, &ns, &tps);
-  if (ns == 1) return 0;
-  const size_t rows = static_cast<size_t>(B) * H * ns * Nq;
-  return align256(rows * d * sizeof(float)) + align256(rows * sizeof(float));
+// Workspace: prefix [B + 1] int64 | bad-length flag | records rec_o
+// [G][2][Nq][d] fp32 | rec_lse [G][2][Nq] fp32, each part 256-byte aligned.
+// It depends on B, Nq and d only.
+struct DecodeWs {
+  size_t prefix, bad, rec_o, rec_lse, total;
+};
+DecodeWs decode_ws_layout(int B, int Nq, int d) {
+  DecodeWs w;
+  const size_t recs = static_cast<size_t>(fa::kDecodeGrid) * 2 * Nq;
+  w.prefix = 0;
+  w.bad = align256((static_cast<size_t>(B) + 1) * sizeof(long long));
+  w.rec_o = w.bad + 256;
+  w.rec_lse = w.rec_o + align256(recs * d * sizeof(float));
+  w.total = w.rec_lse + align256(recs * sizeof(float));
+  return w;
 }
 
 template <int D, int NQ>
 fa_status launch_decode(int dev, const CUtensorMap& mk, const CUtensorMap& mv, const fa::DecParams& p,
                         cudaStream_t s) {
   static bool done[kMaxDevices] = {};
-  auto kern = fa::fa_decode_split_kernel<D, NQ>;
+  auto kern = fa::fa_decode_stream_kernel<D, NQ>;
   constexpr int smem = fa::DecCfg<D, NQ>::SMEM_BYTES;
-  static_assert(fa::DecCfg<D, NQ>::KT == kDecodeTileKeys, "tile size of the split choice");
   fa_status st = ensure_smem(kern, dev, smem, done);
   if (st != FA_OK) return st;
-  kern<<<dim3(static_cast<unsigned>(p.nsplit), static_cast<unsigned>(p.H), static_cast<unsigned>(p.B)),
-         fa::DecCfg<D, NQ>::THREADS, smem, s>>>(mk, mv, p);
+  fa::fa_decode_prefix_kernel<<<1, 256, 0, s>>>(p);
   if ((st = launch_status()) != FA_OK) return st;
-  if (p.nsplit > 1) {
-    const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Nq;
-    fa::fa_decode_merge_kernel<D><<<static_cast<unsigned>((rows + 3) / 4), 128, 0, s>>>(p);
-    if ((st = launch_status()) != FA_OK) return st;
-  }
-  return FA_OK;
+  kern<<<static_cast<unsigned>(p.grid), fa::DecCfg<D, NQ>::THREADS, smem, s>>>(mk, mv, p);
+  if ((st = launch_status()) != FA_OK) return st;
+  const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Nq;
+  fa::fa_decode_merge_kernel_impl<<<static_cast<unsigned>((rows + 3) / 4), 128, 4 * p.grid * sizeof(float), s>>>(p, D);
+  return launch_status();
 }
 
 bool valid_cu(const int* cu, int nseq, int total, int max_seqlen) {
@@ -499,7 +478,7 @@ fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* 
 
 size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d) {
   if (B < 1 || Nq < 1 || Nq > 16 || Nk < 1 || H < 1 || (d != 64 && d != 128)) return 0;
-  return decode_ws_bytes(B, Nq, Nk, H, d);
+  return decode_ws_layout(B, Nq, d).total;
 }
 
 fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
@@ -516,15 +495,15 @@ fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
   if (!std::isfinite(scale)) return FA_ERR_INVALID_ARG;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (static_cast<int64_t>(B) * Nk * H * d > (int64_t(1) << 40)) return FA_ERR_INVALID_ARG;
-  const size_t need = decode_ws_bytes(B, Nq, Nk, H, d);
-  if (need > 0 && (!workspace || ws_bytes < need)) return FA_ERR_WORKSPACE;
-  if (need > 0 && (reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
+  const DecodeWs wl = decode_ws_layout(B, Nq, d);
+  if (!workspace || ws_bytes < wl.total) return FA_ERR_WORKSPACE;
+  if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
   int dev;
   fa_status st = current_device(&dev);
   if (st != FA_OK) return st;
   CUtensorMap mk, mv;
-  if ((st = make_map_bf16(&mk, k_cache, d, H, Nk, B, kDecodeTileKeys)) != FA_OK) return st;
-  if ((st = make_map_bf16(&mv, v_cache, d, H, Nk, B, kDecodeTileKeys)) != FA_OK) return st;
+  if ((st = make_map_bf16(&mk, k_cache, d, H, Nk, B, 64)) != FA_OK) return st;  // 64-key tiles
+  if ((st = make_map_bf16(&mv, v_cache, d, H, Nk, B, 64)) != FA_OK) return st;
   fa::DecParams p;
   p.q = q;
   p.o = o;
@@ -534,11 +513,12 @@ fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache,
   p.Nq = Nq;
   p.Nk = Nk;
   p.H = H;
-  decode_split(B, H, Nk, &p.nsplit, &p.tiles_per_split);
-  const size_t rows = static_cast<size_t>(B) * H * p.nsplit * Nq;
-  p.part_o = p.nsplit > 1 ? static_cast<float*>(workspace) : nullptr;
-  p.part_lse = p.nsplit > 1 ? reinterpret_cast<float*>(static_cast<char*>(workspace) + align256(rows * d * sizeof(float)))
-                            : nullptr;
+  char* ws = static_cast<char*>(workspace);
+  p.prefix = reinterpret_cast<long long*>(ws + wl.prefix);
+  p.bad = reinterpret_cast<int*>(ws + wl.bad);
+  p.rec_o = reinterpret_cast<float*>(ws + wl.rec_o);
+  p.rec_lse = reinterpret_cast<float*>(ws + wl.rec_lse);
+  p.grid = fa::kDecodeGrid;
   p.causal = causal;
   p.scale_log2 = scale * kLog2e;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);

@@ -143,27 +143,30 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_
                      float descale_v, void* o, float* lse, void* workspace, size_t ws_bytes,
                      int B, int N, int H, int d, float scale, int causal, void* stream);
 
-/* Bytes of workspace fa_decode_fwd needs for these sizes (fp32 partial
- * outputs and logsumexps of the key ranges, 256-byte aligned).  0 when the
- * sizes need none (one key range covers the cache) or are invalid. */
+/* Bytes of workspace fa_decode_fwd needs (per-entry tile offsets and fp32
+ * partial outputs and logsumexps of cache segments shared by two or more
+ * CTAs; 256-byte aligned; it depends on B, Nq and d only).  0 for invalid
+ * sizes. */
 size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d);
 
 /* Decode-shaped forward: Nq new queries per batch entry (1 <= Nq <= 16)
  * against a cache of up to Nk keys and values.  The method's tiling and
  * online softmax ("FlashAttention: Fast and Memory-Efficient Exact
  * Attention with IO-Awareness", sections "Tiling" and "Softmax en linea")
- * applied over ranges of the cache in parallel, the ranges merged exactly
- * through their logsumexps.
+ * applied over equal shares of all the cache tiles in parallel (one share
+ * per CTA, whatever the per-sequence lengths), the pieces of a sequence that
+ * falls on several shares merged exactly through their logsumexps.
  * q, o: bf16 [B, Nq, H, d]; k_cache, v_cache: bf16 [B, Nk, H, d];
  * lse: fp32 [B, H, Nq] output (natural log).
  * seqlens_k: int32 device array [B] of valid cache rows per batch entry
  * (0 <= L_b <= Nk), or NULL for all Nk; rows past L_b are never used in the
- * arithmetic (they may hold anything).  A value outside [0, Nk] is reported
- * by fa_get_device_error() and that entry's outputs are not written.
+ * arithmetic (they may hold anything).  If any value is outside [0, Nk]
+ * the call writes no output and fa_get_device_error() reports
+ * FA_ERR_INVALID_ARG.
  * causal = 1: query i is the token at position L_b - Nq + i and sees keys
  * j <= L_b - Nq + i; a query that sees no key gets O = 0 and LSE = -inf.
  * workspace: device buffer of ws_bytes >= fa_decode_workspace_size(...),
- * 256-byte aligned (may be NULL when that size is 0).
+ * 256-byte aligned.
  * Returns FA_ERR_UNSUPPORTED for Nq > 16 or d not in {64, 128}, and
  * FA_ERR_INVALID_ARG for B or H above 65535 (the launch grid's limits). */
 fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,

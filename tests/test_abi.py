@@ -70,7 +70,8 @@ def test_host_validation(L):
     assert L.fa_varlen_bwd_deterministic(*args, ws, P + 2, 1, 8, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
     # decode: q, k, v, o, lse, seqlens, workspace, ws_bytes, B, Nq, Nk, H, d, scale, causal, stream
     dws = fa.decode_workspace_size(1, 1, 16384, 1, 128)
-    assert dws > 0 and fa.decode_workspace_size(64, 1, 300, 16, 128) == 0
+    assert dws > 0 and fa.decode_workspace_size(64, 1, 300, 16, 128) > 0
+    assert fa.decode_workspace_size(1, 1, 16384, 1, 128) == fa.decode_workspace_size(1, 1, 64, 1, 128)  # not Nk
     assert fa.decode_workspace_size(1, 17, 100, 1, 128) == 0 and fa.decode_workspace_size(1, 1, 100, 1, 96) == 0
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 17, 64, 1, 64, 1.0, 0, None) == fa.FA_ERR_UNSUPPORTED
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 1, 64, 1, 96, 1.0, 0, None) == fa.FA_ERR_UNSUPPORTED
@@ -78,6 +79,8 @@ def test_host_validation(L):
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 1, 0, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_decode_fwd(None, P, P, P, P, None, None, 0, 1, 1, 64, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 1, 1, 16384, 1, 128, 1.0, 0, None) == fa.FA_ERR_WORKSPACE
+    assert L.fa_decode_fwd(P, P, P, P, P, None, P * 64, dws - 1, 1, 1, 16384, 1, 128, 1.0, 0, None) == \
+        fa.FA_ERR_WORKSPACE
     assert L.fa_decode_fwd(P, P, P, P, P, None, P + 16, dws, 1, 1, 16384, 1, 128, 1.0, 0, None) == \
         fa.FA_ERR_INVALID_ARG  # workspace not 256-aligned
     assert L.fa_decode_fwd(P, P, P, P, P, None, None, 0, 65536, 1, 64, 1, 64, 1.0, 0, None) == fa.FA_ERR_INVALID_ARG
