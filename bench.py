@@ -65,9 +65,12 @@ def load_peaks():
 
 
 def kernel_source_sha() -> str:
+    """Hash of every file the library is compiled from (the build's own list)."""
+    from exact_io_aware_95_b200 import build as fabuild
     h = hashlib.sha256()
-    for f in ("fa_bwd.cuh", "fa_fwd.cuh", "sm100_ptx.cuh", "fa_api.cu"):
-        with open(os.path.join(ROOT, "exact_io_aware_95_b200", "csrc", f), "rb") as fh:
+    for f in fabuild.deps():
+        with open(f, "rb") as fh:
+            h.update(os.path.relpath(f, ROOT).encode())
             h.update(fh.read())
     return h.hexdigest()[:16]
 
@@ -145,6 +148,29 @@ def cpu_cores() -> int:
         return len(os.sched_getaffinity(0))
     except Exception:
         return os.cpu_count() or 1
+
+
+def host_info() -> dict:
+    """The host the oracle runs on: logical CPUs, the BLAS library's thread
+    count (its matrix products use them all) and the CPU model."""
+    info = {"logical_cpus": os.cpu_count()}
+    try:
+        from threadpoolctl import threadpool_info
+        blas = [p for p in threadpool_info() if p.get("user_api") == "blas"]
+        info["blas_threads"] = max(p["num_threads"] for p in blas) if blas else None
+        info["blas"] = blas[0].get("internal_api") if blas else None
+    except Exception:
+        info["blas_threads"] = None
+    model = None
+    try:
+        for line in open("/proc/cpuinfo"):
+            if line.lower().startswith("model name"):
+                model = line.split(":", 1)[1].strip()
+                break
+    except Exception:
+        pass
+    info["cpu_model"] = model
+    return info
 
 
 _SAMPLE_CACHE = {}
@@ -231,7 +257,7 @@ def run_reference(args, world, rank):
             "scaling": "weak", "vs_baseline": None, "dtype": "f64", "data": "synthetic",
             "config": {"workload": WORKLOAD, "B": w.B, "N": w.N, "H": w.H, "d": w.d, "causal": True},
             "cpu_baseline": {"value": value, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle",
-                             "sample": desc + " per step"},
+                             "sample": desc + " per step", **host_info()},
             "e2e": {"value": value, "unit": UNIT, "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0}}
     return line
 
@@ -261,8 +287,14 @@ def run_gpu(args, world, rank, local):
     fa.check_device_error()
     torch.cuda.synchronize(dev)
 
-    # ---- timed region: whole steps, plus per-call events for the per-kernel roofline
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(3)] for _ in range(args.steps)]
+    # ---- timed region: whole steps, plus per-kernel events for the roofline.
+    # ev[i][0..1] bracket the forward kernel; the library itself records
+    # kev[i][0..3] on the same stream around the three launches of fa_bwd
+    # (preprocess, fused main kernel, dQ conversion).
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(2)] for _ in range(args.steps)]
+    kev = [[torch.cuda.Event(enable_timing=True) for _ in range(4)] for _ in range(args.steps)]
+    for e in (x for row in ev + kev for x in row):
+        e.record(stream)  # torch creates events lazily; the library needs live handles
     t_start, t_end = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
     clocks = ClockSampler(local)
     barrier(world)
@@ -273,8 +305,8 @@ def run_gpu(args, world, rank, local):
         ev[i][0].record(stream)
         fa.fwd(g["q"], g["k"], g["v"], causal=causal, scale=scale, out=o, lse=lse)
         ev[i][1].record(stream)
+        fa.record_launch_events(kev[i])
         fa.bwd(g["q"], g["k"], g["v"], o, lse, g["do"], causal=causal, scale=scale, workspace=ws, dq=dq, dk=dk, dv=dv)
-        ev[i][2].record(stream)
     t_end.record(stream)
     torch.cuda.synchronize(dev)
     barrier(world)
@@ -282,7 +314,9 @@ def run_gpu(args, world, rank, local):
     fa.check_device_error()
     total_ms = allmax(t_start.elapsed_time(t_end), world)
     fwd_ms = statistics.mean(e[0].elapsed_time(e[1]) for e in ev)
-    bwd_ms = statistics.mean(e[1].elapsed_time(e[2]) for e in ev)
+    bwd_ms = statistics.mean(e[0].elapsed_time(e[3]) for e in kev)
+    bwd_stage_ms = [statistics.mean(e[j].elapsed_time(e[j + 1]) for e in kev) for j in range(3)]
+    bwd_main_ms = bwd_stage_ms[1]
     ms_step = total_ms / args.steps
 
     ff = fwd_flops(B, N, H, d, causal)
@@ -290,6 +324,7 @@ def run_gpu(args, world, rank, local):
     value = aggregate_tflops(ff + bf, world, ms_step)
     fwd_tflops = ff / (fwd_ms * 1e-3) / 1e12
     bwd_tflops = bf / (bwd_ms * 1e-3) / 1e12
+    bwd_main_tflops = bf / (bwd_main_ms * 1e-3) / 1e12
     peaks = load_peaks()
 
     # ---- end to end through the public API with pinned host buffers.  Every
@@ -365,15 +400,23 @@ def run_gpu(args, world, rank, local):
                          "fwd_vs_burst": fwd_tflops / peaks["bf16_tflops"],
                          "bwd_vs_burst": bwd_tflops / peaks["bf16_tflops"],
                          "peak_source": peaks["source"]},
-        "roofline": {"kernel": "fa_bwd_kernel (timed as the whole fa_bwd call: preprocess + main + dq_convert)",
-                     "bound": "tensor",
-                     "achieved": bwd_tflops, "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                     "frac": bwd_tflops / peaks["bf16_tflops_sustained"],
-                     "peak_kind": f"sustained bf16 GEMM ({peaks['source']})",
+        "bwd_kernel_ms": {"fa_bwd_preprocess_kernel": bwd_stage_ms[0], "fa_bwd_kernel": bwd_stage_ms[1],
+                          "fa_bwd_dq_convert_kernel": bwd_stage_ms[2]},
+        "roofline": {"kernel": "fa_bwd_kernel", "bound": "tensor",
+                     "achieved": bwd_main_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                     "frac": bwd_main_tflops / peaks["bf16_tflops"],
+                     "peak_kind": f"burst bf16 GEMM ({peaks['source']})",
+                     "how": "687.2 GFLOP (2.5 x the causal forward) per launch / mean CUDA-event duration of the "
+                            "fa_bwd_kernel launch alone, events recorded by the library on the launch stream",
+                     "frac_of_sustained": bwd_main_tflops / peaks["bf16_tflops_sustained"],
                      "traffic": recorded_traffic("fa_bwd_kernel")},
+        "roofline_bwd_call": {"kernels": "fa_bwd call: preprocess + fa_bwd_kernel + dq_convert", "bound": "tensor",
+                              "achieved": bwd_tflops, "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                              "frac": bwd_tflops / peaks["bf16_tflops"]},
         "roofline_fwd": {"kernel": "fa_fwd_kernel", "bound": "tensor", "achieved": fwd_tflops,
-                         "peak": peaks["bf16_tflops_sustained"], "unit": "TFLOP/s",
-                         "frac": fwd_tflops / peaks["bf16_tflops_sustained"],
+                         "peak": peaks["bf16_tflops"], "unit": "TFLOP/s",
+                         "frac": fwd_tflops / peaks["bf16_tflops"],
+                         "frac_of_sustained": fwd_tflops / peaks["bf16_tflops_sustained"],
                          "traffic": recorded_traffic("fa_fwd_kernel")},
         "e2e": {"value": e2e_value, "unit": UNIT, "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h,
                 "ms_per_step": e2e_ms, "steps": e_steps,
@@ -384,7 +427,7 @@ def run_gpu(args, world, rank, local):
     if not args.no_cpu_baseline and world == 1:
         v, dt, desc = oracle_sample(w, 16)  # about 10 s of fp64 work on the host
         line["cpu_baseline"] = {"value": v, "unit": UNIT, "cores": cpu_cores(), "kind": "oracle", "sample": desc,
-                                "seconds": dt}
+                                "seconds": dt, **host_info()}
     return line
 
 
@@ -497,6 +540,51 @@ def run_sweep(args):
         del x
 
 
+def run_oracle_timings(args):
+    """The fp64 oracle timed on the host cores, per workload, mode and
+    direction: full runs where they take seconds to a minute (the tiny, d = 64
+    and Q,K-doubled workloads), else heads {0, H/2, H-1} timed and the time
+    scaled by H/3, labelled as such.  One JSON line each, with the host's
+    cores, BLAS threads and CPU model."""
+    import numpy as np
+    import oracle  # test infrastructure: only the baseline legs call it
+
+    info = host_info()
+    for name, w in WORKLOADS.items():
+        full = (w.varlen_total == 0 and w.N <= 4096)
+        heads = list(range(w.H)) if full else sorted({0, w.H // 2, w.H - 1})
+        x = make_workload(w, seed=args.seed)
+        a = {k: x[k].float().numpy().astype(np.float64) for k in ("q", "k", "v", "do") if k in x}
+        scale = 1.0 / math.sqrt(w.d)
+        for causal in w.causal:
+            if w.varlen_total:
+                lens = x["lengths"]
+                cu = x["cu_seqlens"].numpy()
+                ff = sum(4.0 * w.H * L * L * w.d for L in lens) / (2 if causal else 1)
+                fwd = lambda: oracle.attn_varlen_fwd_ref(a["q"], a["k"], a["v"], cu, scale, causal, heads=heads)
+                bwd = lambda: oracle.attn_varlen_bwd_ref(a["q"], a["k"], a["v"], a["do"], cu, scale, causal,
+                                                         heads=heads)
+                nh = w.H
+            else:
+                ff = fwd_flops(w.B, w.N, w.H, w.d, causal)
+                pairs = [(b, h) for b in range(w.B) for h in heads]
+                fwd = lambda: oracle.attn_fwd_ref(a["q"], a["k"], a["v"], scale, causal, heads=pairs)
+                bwd = lambda: oracle.attn_bwd_ref(a["q"], a["k"], a["v"], a["do"], scale, causal, heads=pairs)
+                nh = w.H
+            dirs = [("fwd", fwd, ff)] + ([("bwd", bwd, 2.5 * ff)] if w.backward else [])
+            for direction, fn, flops in dirs:
+                t0 = time.perf_counter()
+                fn()
+                dt = time.perf_counter() - t0
+                scaled = dt * nh / len(heads)
+                print(json.dumps({
+                    "oracle_timing": name, "causal": causal, "direction": direction,
+                    "heads_timed": len(heads), "heads_total": nh,
+                    "measured_s": dt, "whole_workload_s": scaled,
+                    "kind": "full run" if len(heads) == nh else f"measured on {len(heads)} heads, x{nh}/{len(heads)} extrapolated",
+                    "tflops": flops / scaled / 1e12, "gflop": flops / 1e9, "cores": cpu_cores(), **info}), flush=True)
+
+
 def _sweep_decode(fa, w, args, dev, stream, peaks, iters):
     """Decode lines: HBM-bound, reported as GB/s of the bytes the call must
     move (the valid K and V cache rows, q, o and lse) against the measured
@@ -548,7 +636,12 @@ def main():
     ap.add_argument("--sweep", action="store_true", help="per-call timing of every workload (one GPU)")
     ap.add_argument("--only", default=None, help="with --sweep: one workload by name")
     ap.add_argument("--calls", type=int, default=30, help="with --sweep: timed calls per line (>= 30)")
+    ap.add_argument("--oracle-timings", action="store_true",
+                    help="time the fp64 oracle on the host cores for every workload (no GPU)")
     args = ap.parse_args()
+    if args.oracle_timings:
+        run_oracle_timings(args)
+        return
     if args.sweep:
         run_sweep(args)
         return

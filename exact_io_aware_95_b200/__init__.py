@@ -19,7 +19,7 @@ from typing import Optional, Tuple
 import torch
 
 __all__ = ["FaError", "lib", "fwd", "bwd", "varlen_fwd", "varlen_bwd", "workspace_size", "check_device_error",
-           "decode_fwd", "decode_workspace_size", "fwd_fp8", "fwd_fp8_workspace_size",
+           "decode_fwd", "decode_workspace_size", "fwd_fp8", "fwd_fp8_workspace_size", "record_launch_events",
            "FA_OK", "FA_ERR_INVALID_ARG", "FA_ERR_UNSUPPORTED", "FA_ERR_CUDA", "FA_ERR_TIMEOUT", "FA_ERR_WORKSPACE",
            "EXPORTS", "LIB_PATH"]
 
@@ -47,6 +47,7 @@ EXPORTS = {
     "fa_fwd_fp8": (_I, [_P, _P, _P, _F, _F, _F, _P, _P, _P, _S, _I, _I, _I, _I, _F, _I, _P]),
     "fa_decode_fwd": (_I, [_P, _P, _P, _P, _P, _P, _P, _S, _I, _I, _I, _I, _I, _F, _I, _P]),
     "fa_bwd_noalloc": (_I, [_P, _P, _P, _P, _P, _P, _P, _P, _P, _I, _I, _I, _I, _F, _I, _P]),
+    "fa_record_launch_events": (_I, [ctypes.POINTER(ctypes.c_void_p), _I]),
     "fa_status_string": (ctypes.c_char_p, [_I]),
     "fa_get_device_error": (_I, [_P]),
 }
@@ -105,15 +106,35 @@ def _need(t: torch.Tensor, name: str, dtype, ndim: int):
         raise TypeError(f"{name} must be {dtype}, got {t.dtype}")
     if t.dim() != ndim:
         raise ValueError(f"{name} must have {ndim} dims, got shape {tuple(t.shape)}")
-    if not t.is_cuda:
-        raise ValueError(f"{name} must be on a CUDA device")
     if not t.is_contiguous():
         raise ValueError(f"{name} must be contiguous")
 
 
+def _need_shape(t, name: str, dtype, shape):
+    """`t` must be a contiguous tensor of `dtype` and exactly `shape`:
+    the kernels index every buffer from the sizes of q, so a smaller one
+    would be read or written past its end."""
+    _need(t, name, dtype, len(shape))
+    if tuple(t.shape) != tuple(shape):
+        raise ValueError(f"{name} must have shape {tuple(shape)}, got {tuple(t.shape)}")
+
+
+def _need_workspace(ws, need: int):
+    if not isinstance(ws, torch.Tensor):
+        raise TypeError("workspace must be a torch.Tensor")
+    if not ws.is_contiguous():
+        raise ValueError("workspace must be contiguous")
+    if ws.numel() * ws.element_size() < need:
+        raise FaError(FA_ERR_WORKSPACE, f"workspace of {ws.numel() * ws.element_size()} bytes < {need} needed")
+
+
 def _same_device(*ts):
+    """Every tensor on one CUDA device (checked after dtypes and shapes, right
+    before the call)."""
     dev = ts[0].device
-    for t in ts[1:]:
+    for t in ts:
+        if not t.is_cuda:
+            raise ValueError(f"all tensors must be on a CUDA device; got one on {t.device}")
         if t.device != dev:
             raise ValueError(f"all tensors must be on {dev}; got one on {t.device}")
 
@@ -136,8 +157,8 @@ def fwd(q: torch.Tensor, k: torch.Tensor, v: torch.Tensor, causal: bool = False,
     B, N, H, d = q.shape
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, N), dtype=torch.float32, device=q.device) if lse is None else lse
-    _need(o, "out", torch.bfloat16, 4)
-    _need(l, "lse", torch.float32, 3)
+    _need_shape(o, "out", torch.bfloat16, q.shape)
+    _need_shape(l, "lse", torch.float32, (B, H, N))
     _same_device(q, k, v, o, l)
     with _on(q):
         st = lib().fa_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(), B, N, H, d,
@@ -152,15 +173,19 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None
 
     deterministic=True: bitwise reproducible gradients (fa_bwd_deterministic:
     dQ summed in a fixed order by a second pass instead of fp32 atomics)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
-        _need(t, n, torch.bfloat16, 4)
-    _need(lse, "lse", torch.float32, 3)
+    _need(q, "q", torch.bfloat16, 4)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need_shape(t, n, torch.bfloat16, q.shape)
     B, N, H, d = q.shape
+    _need_shape(lse, "lse", torch.float32, (B, H, N))
     ws_need = workspace_size(B, N, H, d)
     ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need_shape(t, n, torch.bfloat16, q.shape)
+    _need_workspace(ws, ws_need)
     _same_device(q, k, v, o, lse, do, ws, dq, dk, dv)
     with _on(q):
         fn = lib().fa_bwd_deterministic if deterministic else lib().fa_bwd
@@ -174,13 +199,16 @@ def bwd(q, k, v, o, lse, do, causal: bool = False, scale: Optional[float] = None
 def varlen_fwd(q, k, v, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = False,
                scale: Optional[float] = None, out=None, lse=None):
     """Packed forward: q, k, v [total, H, d]; returns O [total, H, d], LSE [H, total]."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v")):
-        _need(t, n, torch.bfloat16, 3)
+    _need(q, "q", torch.bfloat16, 3)
+    for t, n in ((k, "k"), (v, "v")):
+        _need_shape(t, n, torch.bfloat16, q.shape)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
     total, H, d = q.shape
     nseq = cu_seqlens.numel() - 1
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((H, total), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need_shape(o, "out", torch.bfloat16, q.shape)
+    _need_shape(l, "lse", torch.float32, (H, total))
     _same_device(q, k, v, o, l, cu_seqlens)
     with _on(q):
         st = lib().fa_varlen_fwd(q.data_ptr(), k.data_ptr(), v.data_ptr(), o.data_ptr(), l.data_ptr(),
@@ -193,17 +221,21 @@ def varlen_fwd(q, k, v, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool 
 def varlen_bwd(q, k, v, o, lse, do, cu_seqlens: torch.Tensor, max_seqlen: int, causal: bool = False,
                scale: Optional[float] = None, workspace=None, dq=None, dk=None, dv=None, deterministic: bool = False):
     """Packed backward; deterministic=True as for bwd (fa_varlen_bwd_deterministic)."""
-    for t, n in ((q, "q"), (k, "k"), (v, "v"), (o, "o"), (do, "do")):
-        _need(t, n, torch.bfloat16, 3)
-    _need(lse, "lse", torch.float32, 2)
+    _need(q, "q", torch.bfloat16, 3)
+    for t, n in ((k, "k"), (v, "v"), (o, "o"), (do, "do")):
+        _need_shape(t, n, torch.bfloat16, q.shape)
     _need(cu_seqlens, "cu_seqlens", torch.int32, 1)
     total, H, d = q.shape
+    _need_shape(lse, "lse", torch.float32, (H, total))
     nseq = cu_seqlens.numel() - 1
     ws_need = workspace_size(1, total, H, d)
     ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device) if workspace is None else workspace
     dq = torch.empty_like(q) if dq is None else dq
     dk = torch.empty_like(k) if dk is None else dk
     dv = torch.empty_like(v) if dv is None else dv
+    for t, n in ((dq, "dq"), (dk, "dk"), (dv, "dv")):
+        _need_shape(t, n, torch.bfloat16, q.shape)
+    _need_workspace(ws, ws_need)
     _same_device(q, k, v, o, lse, do, cu_seqlens, ws, dq, dk, dv)
     with _on(q):
         fn = lib().fa_varlen_bwd_deterministic if deterministic else lib().fa_varlen_bwd
@@ -233,7 +265,9 @@ def fwd_fp8(q, k, v, descale_q: float, descale_k: float, descale_v: float, causa
     ws = workspace
     if ws is None:
         ws = torch.empty(max(fwd_fp8_workspace_size(B, N, H, d), 256), dtype=torch.uint8, device=q.device)
-    _need(o, "out", torch.bfloat16, 4)
+    _need_shape(o, "out", torch.bfloat16, q.shape)
+    _need_shape(l, "lse", torch.float32, (B, H, N))
+    _need_workspace(ws, fwd_fp8_workspace_size(B, N, H, d))
     _same_device(q, k, v, o, l, ws)
     with _on(q):
         st = lib().fa_fwd_fp8(q.data_ptr(), k.data_ptr(), v.data_ptr(), float(descale_q), float(descale_k),
@@ -266,10 +300,14 @@ def decode_fwd(q, k_cache, v_cache, seqlens_k: Optional[torch.Tensor] = None, ca
             raise ValueError("seqlens_k must have B entries")
     o = torch.empty_like(q) if out is None else out
     l = torch.empty((B, H, Nq), dtype=torch.float32, device=q.device) if lse is None else lse
+    _need_shape(o, "out", torch.bfloat16, q.shape)
+    _need_shape(l, "lse", torch.float32, (B, H, Nq))
     ws_need = decode_workspace_size(B, Nq, Nk, H, d)
     ws = workspace
     if ws is None and ws_need > 0:
         ws = torch.empty(ws_need, dtype=torch.uint8, device=q.device)
+    if ws is not None:
+        _need_workspace(ws, ws_need)
     ts = [q, k_cache, v_cache, o, l] + [t for t in (seqlens_k, ws) if t is not None]
     _same_device(*ts)
     with _on(q):
@@ -280,6 +318,18 @@ def decode_fwd(q, k_cache, v_cache, seqlens_k: Optional[torch.Tensor] = None, ca
                                  B, Nq, Nk, H, d, _scale(scale, d), int(bool(causal)), _stream_ptr(q))
     _check(st, "fa_decode_fwd")
     return o, l
+
+
+def record_launch_events(events):
+    """Measurement hook: the next library call made by this thread records the
+    given torch.cuda.Event objects on its stream, events[0] before its first
+    kernel launch and events[i] after its i-th launch.  Each event must have
+    been recorded once already (so that torch has created it)."""
+    handles = [int(e.cuda_event) for e in events]
+    if not all(handles):
+        raise ValueError("record each event once before passing it (torch creates events lazily)")
+    arr = (ctypes.c_void_p * len(handles))(*handles)
+    _check(lib().fa_record_launch_events(arr, len(handles)), "fa_record_launch_events")
 
 
 def check_device_error(stream: Optional[torch.cuda.Stream] = None):

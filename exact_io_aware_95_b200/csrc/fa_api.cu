@@ -168,9 +168,30 @@ fa_status make_map_u8(CUtensorMap* m, const void* base, const uint64_t (&dims)[4
   return r == CUDA_SUCCESS ? FA_OK : FA_ERR_CUDA;
 }
 
-fa_status launch_status() {
+// Measurement hook (fa_record_launch_events): caller-created CUDA events that
+// the next compute call of this host thread records between its launches.
+struct LaunchEvents {
+  cudaEvent_t ev[8];
+  int n = 0;
+  int used = 0;
+};
+thread_local LaunchEvents t_launch_events;
+
+void mark_launch(cudaStream_t s) {
+  LaunchEvents& h = t_launch_events;
+  if (h.used < h.n && cudaEventRecord(h.ev[h.used], s) == cudaSuccess) ++h.used;
+}
+
+// Clears the hook when a public compute call returns, however it returns.
+struct LaunchEventsScope {
+  ~LaunchEventsScope() { t_launch_events.n = t_launch_events.used = 0; }
+};
+
+fa_status launch_status(cudaStream_t s) {
   cudaError_t e = cudaGetLastError();
-  return e == cudaSuccess ? FA_OK : FA_ERR_CUDA;
+  if (e != cudaSuccess) return FA_ERR_CUDA;
+  mark_launch(s);
+  return FA_OK;
 }
 
 constexpr float kLog2e = 1.4426950408889634f;
@@ -197,8 +218,9 @@ fa_status launch_fwd(int dev, const CUtensorMap& q, const CUtensorMap& k, const 
   if (st != FA_OK) return st;
   const int64_t grid = static_cast<int64_t>(p.npairs) * p.B * p.H;
   if (grid <= 0 || grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
+  mark_launch(s);
   kern<<<static_cast<unsigned>(grid), fa::FwdCfg<D, PTM>::THREADS, smem, s>>>(q, k, v, p);
-  return launch_status();
+  return launch_status(s);
 }
 
 template <int D>
@@ -271,14 +293,15 @@ fa_status launch_bwd_det(int dev, const CUtensorMap& mq, const CUtensorMap& mk, 
   {
     const int64_t blocks = (static_cast<int64_t>(p.rows) * p.H + 7) / 8;
     if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    mark_launch(s);
     fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
-    if ((st = launch_status()) != FA_OK) return st;
+    if ((st = launch_status(s)) != FA_OK) return st;
   }
   kmain<<<static_cast<unsigned>(grid), fa::BwdCfg<D>::THREADS, smem_main, s>>>(mq, mk, mv, mdo, p);
-  if ((st = launch_status()) != FA_OK) return st;
+  if ((st = launch_status(s)) != FA_OK) return st;
   p.group = dq_group;
   kdq<<<static_cast<unsigned>(grid), fa::DqCfg<D>::THREADS, smem_dq, s>>>(mq, mk, mv, mdo, p);
-  return launch_status();
+  return launch_status(s);
 }
 
 template <int D, bool CAUSAL, bool VARLEN>
@@ -294,15 +317,16 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
     const int64_t rows = static_cast<int64_t>(p.rows) * p.H;  // one warp per (token, head)
     const int64_t blocks = (rows + 7) / 8;
     if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
+    mark_launch(s);
     fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
-    if ((st = launch_status()) != FA_OK) return st;
+    if ((st = launch_status(s)) != FA_OK) return st;
   }
   // 2) fused recompute + dK, dV, dQ accumulation, one CTA per 128-key tile
   {
     const int64_t grid = static_cast<int64_t>(p.nkvtiles) * p.B * p.H;
     if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
     kern<<<static_cast<unsigned>(grid), fa::BwdCfg<D>::THREADS, smem, s>>>(mq, mk, mv, mdo, p);
-    if ((st = launch_status()) != FA_OK) return st;
+    if ((st = launch_status(s)) != FA_OK) return st;
   }
   // 3) dQ = bf16(scale * dQ accumulator)
   {
@@ -310,7 +334,7 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
     const int64_t blocks = (n8 + 255) / 256;
     if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
     fa::fa_bwd_dq_convert_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
-    if ((st = launch_status()) != FA_OK) return st;
+    if ((st = launch_status(s)) != FA_OK) return st;
   }
   return FA_OK;
 }
@@ -409,13 +433,14 @@ fa_status launch_decode(int dev, const CUtensorMap& mk, const CUtensorMap& mv, c
   constexpr int smem = fa::DecCfg<D, NQ>::SMEM_BYTES;
   fa_status st = ensure_smem(kern, dev, smem, done);
   if (st != FA_OK) return st;
+  mark_launch(s);
   fa::fa_decode_prefix_kernel<<<1, 256, 0, s>>>(p);
-  if ((st = launch_status()) != FA_OK) return st;
+  if ((st = launch_status(s)) != FA_OK) return st;
   kern<<<static_cast<unsigned>(p.grid), fa::DecCfg<D, NQ>::THREADS, smem, s>>>(mk, mv, p);
-  if ((st = launch_status()) != FA_OK) return st;
+  if ((st = launch_status(s)) != FA_OK) return st;
   const int64_t rows = static_cast<int64_t>(p.B) * p.H * p.Nq;
   fa::fa_decode_merge_kernel_impl<<<static_cast<unsigned>((rows + 3) / 4), 128, 4 * p.grid * sizeof(float), s>>>(p, D);
-  return launch_status();
+  return launch_status(s);
 }
 
 bool valid_cu(const int* cu, int nseq, int total, int max_seqlen) {
@@ -428,11 +453,13 @@ extern "C" {
 
 fa_status fa_fwd(const void* q, const void* k, const void* v, void* o, float* lse, int B, int N, int H, int d,
                  float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   return fwd_common(q, k, v, o, lse, nullptr, B, N, N, H, d, scale, causal, stream);
 }
 
 fa_status fa_varlen_fwd(const void* q, const void* k, const void* v, void* o, float* lse, const int* cu_seqlens,
                         int nseq, int total, int max_seqlen, int H, int d, float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
   return fwd_common(q, k, v, o, lse, cu_seqlens, nseq, max_seqlen, total, H, d, scale, causal, stream);
@@ -446,6 +473,7 @@ size_t fa_bwd_workspace_size(int B, int N, int H, int d) {
 fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                  void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B, int N, int H, int d,
                  float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, N, H, d, scale, causal,
                     stream);
 }
@@ -453,6 +481,7 @@ fa_status fa_bwd(const void* q, const void* k, const void* v, const void* o, con
 fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void* o, const float* lse, const void* dO,
                         void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, const int* cu_seqlens,
                         int nseq, int total, int max_seqlen, int H, int d, float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total, H, d,
@@ -462,6 +491,7 @@ fa_status fa_varlen_bwd(const void* q, const void* k, const void* v, const void*
 fa_status fa_bwd_deterministic(const void* q, const void* k, const void* v, const void* o, const float* lse,
                                const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes, int B,
                                int N, int H, int d, float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, nullptr, B, N, N, H, d, scale, causal,
                     stream, true);
 }
@@ -470,6 +500,7 @@ fa_status fa_varlen_bwd_deterministic(const void* q, const void* k, const void* 
                                       const void* dO, void* dq, void* dk, void* dv, void* workspace, size_t ws_bytes,
                                       const int* cu_seqlens, int nseq, int total, int max_seqlen, int H, int d,
                                       float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (!valid_cu(cu_seqlens, nseq, total, max_seqlen)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(cu_seqlens) & 3u) != 0) return FA_ERR_INVALID_ARG;
   return bwd_common(q, k, v, o, lse, dO, dq, dk, dv, workspace, ws_bytes, cu_seqlens, nseq, max_seqlen, total, H, d,
@@ -484,6 +515,7 @@ size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d) {
 fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                         const int* seqlens_k, void* workspace, size_t ws_bytes, int B, int Nq, int Nk, int H, int d,
                         float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (!q || !k_cache || !v_cache || !o || !lse) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k_cache) || !aligned16(v_cache) || !aligned16(o) || !aligned16(lse))
     return FA_ERR_INVALID_ARG;
@@ -535,6 +567,7 @@ size_t fa_fwd_fp8_workspace_size(int B, int N, int H, int d) {
 fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_q, float descale_k, float descale_v,
                      void* o, float* lse, void* workspace, size_t ws_bytes, int B, int N, int H, int d, float scale,
                      int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (!q || !k || !v || !o || !lse || !workspace) return FA_ERR_INVALID_ARG;
   if (!aligned16(q) || !aligned16(k) || !aligned16(v) || !aligned16(o) || !aligned16(lse)) return FA_ERR_INVALID_ARG;
   if ((reinterpret_cast<uintptr_t>(workspace) & 255u) != 0) return FA_ERR_INVALID_ARG;
@@ -570,11 +603,12 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_
   constexpr int smem = fa::Fp8Cfg::SMEM_BYTES;
   if ((st = ensure_smem(kern, dev, smem, causal ? done_c : done_nc, fa::kLaunchRegs)) != FA_OK) return st;
   cudaStream_t s = reinterpret_cast<cudaStream_t>(stream);
+  mark_launch(s);
   fa::fa_fp8_transpose_v_kernel<<<dim3(static_cast<unsigned>((npad + 127) / 128), static_cast<unsigned>(H),
                                        static_cast<unsigned>(B)),
                                   128, 0, s>>>(static_cast<const uint8_t*>(v), static_cast<uint8_t*>(workspace), N,
                                                H, static_cast<int>(npad));
-  if ((st = launch_status()) != FA_OK) return st;
+  if ((st = launch_status(s)) != FA_OK) return st;
   fa::Fp8Params p;
   p.o = o;
   p.lse = lse;
@@ -588,7 +622,18 @@ fa_status fa_fwd_fp8(const void* q, const void* k, const void* v, float descale_
   const int64_t grid = static_cast<int64_t>(p.npairs) * B * H;
   if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
   kern<<<static_cast<unsigned>(grid), fa::Fp8Cfg::THREADS, smem, s>>>(mq, mk, mvt, p);
-  return launch_status();
+  return launch_status(s);
+}
+
+fa_status fa_record_launch_events(void* const* events, int n) {
+  if (!events || n < 1 || n > 8) return FA_ERR_INVALID_ARG;
+  for (int i = 0; i < n; ++i)
+    if (!events[i]) return FA_ERR_INVALID_ARG;
+  LaunchEvents& h = t_launch_events;
+  for (int i = 0; i < n; ++i) h.ev[i] = static_cast<cudaEvent_t>(events[i]);
+  h.n = n;
+  h.used = 0;
+  return FA_OK;
 }
 
 const char* fa_status_string(fa_status s) {
@@ -667,6 +712,7 @@ fa_status static_scratch(int dev, void** out) {
 extern "C" fa_status fa_bwd_noalloc(const void* q, const void* k, const void* v, const void* o, const float* lse,
                                     const void* dO, void* dq, void* dk, void* dv, int B, int N, int H, int d,
                                     float scale, int causal, void* stream) {
+  LaunchEventsScope hook_scope;
   if (d != 64 && d != 128) return FA_ERR_UNSUPPORTED;
   if (B < 1 || N < 1 || H < 1) return FA_ERR_INVALID_ARG;
   const size_t need = fa_bwd_workspace_size(B, N, H, d);

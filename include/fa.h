@@ -36,8 +36,10 @@
  * the launch; errors found on the host are returned before anything is
  * launched.  Calls are thread-safe.
  *
- * Errors.  FA_ERR_INVALID_ARG for a null or misaligned pointer, a size < 1
- * or too large, or a too-small workspace; FA_ERR_UNSUPPORTED for d not in
+ * Errors.  FA_ERR_INVALID_ARG for a null or misaligned pointer or a size < 1
+ * or too large; FA_ERR_WORKSPACE for a workspace smaller than the call needs
+ * (and, in fa_bwd_noalloc, a problem larger than its static scratch);
+ * FA_ERR_UNSUPPORTED for d not in
  * {64, 128} or a device that is not compute capability 10.0 (sm_100); FA_ERR_CUDA
  * when a CUDA call or launch fails.  Every on-device pipeline wait is bounded:
  * an expired wait ends the kernel and sets a device error word, which
@@ -172,6 +174,18 @@ size_t fa_decode_workspace_size(int B, int Nq, int Nk, int H, int d);
 fa_status fa_decode_fwd(const void* q, const void* k_cache, const void* v_cache, void* o, float* lse,
                         const int* seqlens_k, void* workspace, size_t ws_bytes,
                         int B, int Nq, int Nk, int H, int d, float scale, int causal, void* stream);
+
+/* Measurement hook (no counterpart in the method: it serves the roofline
+ * measurement, which times the dominant kernel of a multi-kernel call on its
+ * own).  events: n (1..8) cudaEvent_t handles, created by the caller on the
+ * current device and owned by it.  The NEXT compute call made by this host
+ * thread records events[0] on that call's stream just before its first kernel
+ * launch and events[i] right after its i-th launch, as far as n reaches; the
+ * hook is then cleared, whether that call succeeded or not.  For fa_bwd the
+ * launches are: D / accumulator preprocess, the fused main kernel, the dQ
+ * conversion.  FA_ERR_INVALID_ARG for a null array or entry, or n outside
+ * 1..8.  Recording an event adds no work to the kernels themselves. */
+fa_status fa_record_launch_events(void* const* events, int n);
 
 /* Backward pass, dense batch, for callers that cannot allocate device memory.
  * There is no counterpart to this in the method's description: it exists for

@@ -91,3 +91,12 @@ def test_host_validation(L):
 def test_compute_call_without_gpu_reports_cuda_error(L):
     P = 4096
     assert L.fa_fwd(P, P, P, P, P, 1, 8, 1, 64, 1.0, 0, None) == fa.FA_ERR_CUDA
+
+
+def test_launch_event_hook_validates_on_the_host(L):
+    import ctypes
+    assert L.fa_record_launch_events(None, 1) == fa.FA_ERR_INVALID_ARG
+    arr = (ctypes.c_void_p * 2)(4096, 0)
+    assert L.fa_record_launch_events(arr, 2) == fa.FA_ERR_INVALID_ARG   # null entry
+    assert L.fa_record_launch_events(arr, 0) == fa.FA_ERR_INVALID_ARG
+    assert L.fa_record_launch_events(arr, 9) == fa.FA_ERR_INVALID_ARG

@@ -15,7 +15,7 @@ from exact_io_aware_95_b200 import build as fabuild
 
 HERE = os.path.dirname(os.path.abspath(__file__))
 ROOT = os.path.dirname(HERE)
-CUDA = "/usr/local/cuda"
+CUDA = fabuild.cuda_home()
 
 
 @pytest.fixture(scope="module")
