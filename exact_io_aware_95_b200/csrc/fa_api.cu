@@ -10,10 +10,6 @@
 
 #include "fa.h"
 
-// Forward variant: P through tensor memory (1) or through shared memory (0).
-#ifndef FA_FWD_P_IN_TMEM
-#define FA_FWD_P_IN_TMEM 1
-#endif
 #include "fa_bwd.cuh"
 #include "fa_bwd_dq.cuh"
 #include "fa_decode.cuh"
@@ -211,15 +207,16 @@ template <int D, bool CAUSAL, bool VARLEN>
 fa_status launch_fwd(int dev, const CUtensorMap& q, const CUtensorMap& k, const CUtensorMap& v,
                      const fa::FwdParams& p, cudaStream_t s) {
   static bool done[kMaxDevices] = {};
-  constexpr bool PTM = FA_FWD_P_IN_TMEM;
-  auto kern = fa::fa_fwd_kernel<D, CAUSAL, VARLEN, PTM>;
-  constexpr int smem = fa::FwdCfg<D, PTM>::SMEM_BYTES;
+  auto kern = fa::fa_fwd_kernel<D, CAUSAL, VARLEN>;
+  constexpr int smem = fa::FwdCfg<D>::SMEM_BYTES;
   fa_status st = ensure_smem(kern, dev, smem, done, fa::kLaunchRegs);
   if (st != FA_OK) return st;
+  // one CTA per work item; running CTAs take over the items of CTAs that have
+  // not started (cluster launch control), so about one CTA per SM runs
   const int64_t grid = static_cast<int64_t>(p.npairs) * p.B * p.H;
   if (grid <= 0 || grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
   mark_launch(s);
-  kern<<<static_cast<unsigned>(grid), fa::FwdCfg<D, PTM>::THREADS, smem, s>>>(q, k, v, p);
+  kern<<<static_cast<unsigned>(grid), fa::FwdCfg<D>::THREADS, smem, s>>>(q, k, v, p);
   return launch_status(s);
 }
 

@@ -314,3 +314,69 @@ __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
 }  // namespace fa
+
+namespace fa {
+// ------------------------------------------------------------ packed fp32 pairs
+// sm_100 executes some fp32 arithmetic on register pairs in one instruction
+// (add/mul/fma .f32x2); a pair lives in one 64-bit register, low word first.
+__device__ __forceinline__ uint64_t f2_pack(float lo, float hi) {
+  uint64_t r;
+  asm("mov.b64 %0, {%1, %2};" : "=l"(r) : "f"(lo), "f"(hi));
+  return r;
+}
+__device__ __forceinline__ void f2_unpack(uint64_t v, float& lo, float& hi) {
+  asm("mov.b64 {%0, %1}, %2;" : "=f"(lo), "=f"(hi) : "l"(v));
+}
+__device__ __forceinline__ uint64_t ffma2(uint64_t a, uint64_t b, uint64_t c) {
+  uint64_t d;
+  asm("fma.rn.f32x2 %0, %1, %2, %3;" : "=l"(d) : "l"(a), "l"(b), "l"(c));
+  return d;
+}
+__device__ __forceinline__ uint64_t fadd2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("add.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ uint64_t fmul2(uint64_t a, uint64_t b) {
+  uint64_t d;
+  asm("mul.f32x2 %0, %1, %2;" : "=l"(d) : "l"(a), "l"(b));
+  return d;
+}
+__device__ __forceinline__ float f2_sum(uint64_t v) {
+  float lo, hi;
+  f2_unpack(v, lo, hi);
+  return lo + hi;
+}
+
+// ------------------------------------------------------- cluster launch control
+// A running CTA asks the hardware to cancel the launch of a CTA of the same
+// grid that has not started yet and takes over its work: the grid keeps the
+// hardware's own launch order and load balance, while each running CTA keeps
+// its on-chip set-up (tensor memory, barriers, pipelines) across work items.
+// The 16-byte response lands in shared memory `resp` (16-byte aligned) and
+// completes 16 bytes of transaction on mbarrier `bar`.  After a request that
+// comes back "not cancelled" no further request may be issued.
+__device__ __forceinline__ void clc_try_cancel(uint32_t resp, uint32_t bar) {
+  asm volatile("clusterlaunchcontrol.try_cancel.async.shared::cta.mbarrier::complete_tx::bytes.b128 [%0], [%1];" ::"r"(
+                   resp),
+               "r"(bar)
+               : "memory");
+}
+// blockIdx.x of the cancelled CTA, or -1 when nothing was cancelled.
+__device__ __forceinline__ int clc_query(uint32_t resp) {
+  uint32_t valid, x = 0;
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t.reg .b128 rsp;\n\t"
+      "ld.shared.b128 rsp, [%2];\n\t"
+      "clusterlaunchcontrol.query_cancel.is_canceled.pred.b128 p, rsp;\n\t"
+      "selp.u32 %0, 1, 0, p;\n\t"
+      "@p clusterlaunchcontrol.query_cancel.get_first_ctaid::x.b32.b128 %1, rsp;\n\t}"
+      : "=r"(valid), "=r"(x)
+      : "r"(resp)
+      : "memory");
+  return valid ? static_cast<int>(x) : -1;
+}
+__device__ __forceinline__ void ld_shared_v4(uint32_t addr, uint32_t& a, uint32_t& b, uint32_t& c, uint32_t& d) {
+  asm volatile("ld.shared.v4.b32 {%0, %1, %2, %3}, [%4];" : "=r"(a), "=r"(b), "=r"(c), "=r"(d) : "r"(addr) : "memory");
+}
+}  // namespace fa
