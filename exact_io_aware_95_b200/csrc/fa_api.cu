@@ -264,6 +264,17 @@ fa_status fwd_common(const void* q, const void* k, const void* v, void* o, float
 }
 
 // ----------------------------------------------------------------- backward
+// Grid of the memory-bound preprocess: grid-stride loops over a resident wave
+// (8 blocks of 256 threads per SM).
+unsigned preprocess_blocks(int dev) {
+  int sms = 148;
+  if (cudaDeviceGetAttribute(&sms, cudaDevAttrMultiProcessorCount, dev) != cudaSuccess) {
+    cudaGetLastError();
+    sms = 148;
+  }
+  return static_cast<unsigned>(sms * 8);
+}
+
 size_t align256(size_t x) { return (x + 255) & ~size_t(255); }
 
 size_t ws_bytes_for(int64_t rows, int H, int d) {
@@ -288,10 +299,8 @@ fa_status launch_bwd_det(int dev, const CUtensorMap& mq, const CUtensorMap& mk, 
   const int64_t grid = static_cast<int64_t>(p.nkvtiles) * p.B * p.H;
   if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;
   {
-    const int64_t blocks = (static_cast<int64_t>(p.rows) * p.H + 7) / 8;
-    if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
     mark_launch(s);
-    fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    fa::fa_bwd_preprocess_kernel<D><<<preprocess_blocks(dev), 256, 0, s>>>(p);
     if ((st = launch_status(s)) != FA_OK) return st;
   }
   kmain<<<static_cast<unsigned>(grid), fa::BwdCfg<D>::THREADS, smem_main, s>>>(mq, mk, mv, mdo, p);
@@ -311,11 +320,8 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   if (st != FA_OK) return st;
   // 1) D = rowsum(dO * O) and zeroed dQ accumulator
   {
-    const int64_t rows = static_cast<int64_t>(p.rows) * p.H;  // one warp per (token, head)
-    const int64_t blocks = (rows + 7) / 8;
-    if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
     mark_launch(s);
-    fa::fa_bwd_preprocess_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
+    fa::fa_bwd_preprocess_kernel<D><<<preprocess_blocks(dev), 256, 0, s>>>(p);
     if ((st = launch_status(s)) != FA_OK) return st;
   }
   // 2) fused recompute + dK, dV, dQ accumulation, one CTA per 128-key tile
@@ -327,8 +333,9 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
   }
   // 3) dQ = bf16(scale * dQ accumulator)
   {
-    const int64_t n8 = static_cast<int64_t>(p.rows) * p.H * D / 8;
-    const int64_t blocks = (n8 + 255) / 256;
+    const int64_t R = p.cu_seqlens ? p.total : p.N;
+    const int64_t nbh = p.cu_seqlens ? p.H : static_cast<int64_t>(p.B) * p.H;
+    const int64_t blocks = nbh * ((R + 31) / 32);
     if (blocks > 0x7fffffff) return FA_ERR_INVALID_ARG;
     fa::fa_bwd_dq_convert_kernel<D><<<static_cast<unsigned>(blocks), 256, 0, s>>>(p);
     if ((st = launch_status(s)) != FA_OK) return st;

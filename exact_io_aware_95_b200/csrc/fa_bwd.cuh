@@ -80,80 +80,107 @@ __device__ __forceinline__ size_t dq_acc_index4(int bh, int g, int64_t r, int64_
 }
 
 // ------------------------------------------------------------------ preprocess
-// One warp per (token, head) row computes D; every thread also zeroes one
-// float4 of the accumulator (linear order, layout independent).
+// D_i = sum_c dO_ic O_ic for every (token, head) row, and the fp32 dQ
+// accumulator zeroed.  Memory-bound: each lane reads 16 bytes of O and of dO
+// (a d = 128 row is 16 lanes, so a warp covers 2 rows per step, 4 at d = 64)
+// and the zeroing runs as a separate grid-stride loop of 16-byte stores.
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_preprocess_kernel(const BwdParams p) {
+  constexpr int LPR = D / 8;         // lanes per row (8 bf16 = 16 bytes per lane)
+  constexpr int RPW = 32 / LPR;      // rows per warp step
+  const int64_t nthreads = static_cast<int64_t>(gridDim.x) * blockDim.x;
   const int64_t gtid = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
-  const int64_t nacc4 = static_cast<int64_t>(p.rows) * p.H * (D / 4);
-  if (p.dq_acc && gtid < nacc4) reinterpret_cast<float4*>(p.dq_acc)[gtid] = make_float4(0.f, 0.f, 0.f, 0.f);
-  const int64_t w = gtid >> 5;
-  const int lane = threadIdx.x & 31;
-  const int64_t nrows = static_cast<int64_t>(p.rows) * p.H;
-  if (w >= nrows) return;
-  const int64_t tok = w / p.H;
-  const int h = static_cast<int>(w % p.H);
-  const size_t base = static_cast<size_t>(w) * D;  // [rows, H, D] element offset
-  constexpr int PER = D / 32;                      // elements per lane (2 or 4)
-  const __nv_bfloat16* o = reinterpret_cast<const __nv_bfloat16*>(p.o) + base + lane * PER;
-  const __nv_bfloat16* g = reinterpret_cast<const __nv_bfloat16*>(p.dout) + base + lane * PER;
-  float acc = 0.f;
-  if (PER == 4) {
-    const uint2 ov = *reinterpret_cast<const uint2*>(o);
-    const uint2 gv = *reinterpret_cast<const uint2*>(g);
-    acc = bf16lo_to_f32(ov.x) * bf16lo_to_f32(gv.x) + bf16hi_to_f32(ov.x) * bf16hi_to_f32(gv.x) +
-          bf16lo_to_f32(ov.y) * bf16lo_to_f32(gv.y) + bf16hi_to_f32(ov.y) * bf16hi_to_f32(gv.y);
-  } else {
-    const uint32_t ov = *reinterpret_cast<const uint32_t*>(o);
-    const uint32_t gv = *reinterpret_cast<const uint32_t*>(g);
-    acc = bf16lo_to_f32(ov) * bf16lo_to_f32(gv) + bf16hi_to_f32(ov) * bf16hi_to_f32(gv);
+  if (p.dq_acc) {
+    const int64_t nacc4 = static_cast<int64_t>(p.rows) * p.H * (D / 4);
+    float4* acc = reinterpret_cast<float4*>(p.dq_acc);
+    for (int64_t i = gtid; i < nacc4; i += nthreads) acc[i] = make_float4(0.f, 0.f, 0.f, 0.f);
   }
+  const int lane = threadIdx.x & 31;
+  const int sub = lane / LPR, part = lane % LPR;
+  const int64_t nrows = static_cast<int64_t>(p.rows) * p.H;  // (token, head) rows
+  const int64_t nwarps = nthreads >> 5;
+  constexpr int U = 4;  // warp steps whose loads are in flight together
+  for (int64_t w0 = (gtid >> 5) * U; w0 * RPW < nrows; w0 += nwarps * U) {
+    uint4 ov[U], gv[U];
 #pragma unroll
-  for (int off = 16; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
-  if (lane == 0) {
-    size_t li;
-    if (p.cu_seqlens) {
-      li = static_cast<size_t>(h) * p.total + tok;
-    } else {
-      const int64_t b = tok / p.N, n = tok % p.N;
-      li = (static_cast<size_t>(b) * p.H + h) * p.N + n;
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = (w0 + u) * RPW + sub;
+      if (row < nrows) {
+        const size_t off = static_cast<size_t>(row) * D + part * 8;
+        ov[u] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.o) + off);
+        gv[u] = *reinterpret_cast<const uint4*>(reinterpret_cast<const __nv_bfloat16*>(p.dout) + off);
+      } else {
+        ov[u] = gv[u] = make_uint4(0u, 0u, 0u, 0u);
+      }
     }
-    p.dvec[li] = acc;
+#pragma unroll
+    for (int u = 0; u < U; ++u) {
+      const int64_t row = (w0 + u) * RPW + sub;
+      const uint32_t ow[4] = {ov[u].x, ov[u].y, ov[u].z, ov[u].w}, gw[4] = {gv[u].x, gv[u].y, gv[u].z, gv[u].w};
+      float acc = 0.f;
+#pragma unroll
+      for (int e = 0; e < 4; ++e)
+        acc += bf16lo_to_f32(ow[e]) * bf16lo_to_f32(gw[e]) + bf16hi_to_f32(ow[e]) * bf16hi_to_f32(gw[e]);
+#pragma unroll
+      for (int off = LPR / 2; off > 0; off >>= 1) acc += __shfl_xor_sync(0xffffffffu, acc, off);
+      if (part == 0 && row < nrows) {
+        const int64_t tok = row / p.H;
+        const int h = static_cast<int>(row % p.H);
+        size_t li;
+        if (p.cu_seqlens) {
+          li = static_cast<size_t>(h) * p.total + tok;
+        } else {
+          const int64_t b = tok / p.N, n = tok % p.N;
+          li = (static_cast<size_t>(b) * p.H + h) * p.N + n;
+        }
+        p.dvec[li] = acc;
+      }
+    }
   }
 }
 
 // ------------------------------------------------------------------ dQ convert
-// Thread i handles 8 columns (float4 groups 2k, 2k+1) of one (bh, row):
-// i = (bh * D/8 + k) * R + r, so a warp reads 32 consecutive rows of a group.
+// dQ = bf16(scale * accumulator).  One block per (batch entry or sequence
+// head, 32 consecutive query rows): the column-block-major accumulator is read
+// as 512-byte runs (32 rows of one 4-column group per warp), transposed through
+// shared memory, and written as whole rows (D * 2 contiguous bytes per row).
 template <int D>
 __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams p) {
-  const int64_t i = static_cast<int64_t>(blockIdx.x) * blockDim.x + threadIdx.x;
+  constexpr int G = D / 4;  // float4 groups per row
+  __shared__ float4 tile[32][G + 1];
   const int64_t R = p.cu_seqlens ? p.total : p.N;
-  const int64_t nbh = p.cu_seqlens ? p.H : static_cast<int64_t>(p.B) * p.H;
-  if (i >= nbh * (D / 8) * R) return;
-  const int64_t r = i % R;
-  const int64_t t = i / R;
-  const int k = static_cast<int>(t % (D / 8));
-  const int bh = static_cast<int>(t / (D / 8));
+  const int64_t nblk = (R + 31) / 32;
+  const int bh = static_cast<int>(blockIdx.x / nblk);
+  const int64_t r0 = (blockIdx.x % nblk) * 32;
+  const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const float4* acc = reinterpret_cast<const float4*>(p.dq_acc);
-  const float4 a = acc[dq_acc_index4(bh, 2 * k, r, R, D)];
-  const float4 c = acc[dq_acc_index4(bh, 2 * k + 1, r, R, D)];
-  int64_t tok;
+#pragma unroll
+  for (int g = w; g < G; g += 8)
+    if (r0 + lane < R) tile[lane][g] = acc[dq_acc_index4(bh, g, r0 + lane, R, D)];
+  __syncthreads();
   int h;
+  int64_t tok0;
   if (p.cu_seqlens) {
     h = bh;
-    tok = r;
+    tok0 = r0;
   } else {
     h = bh % p.H;
-    tok = static_cast<int64_t>(bh / p.H) * p.N + r;
+    tok0 = static_cast<int64_t>(bh / p.H) * p.N + r0;
   }
+  constexpr int CPR = D / 8;  // 16-byte output chunks per row
   const float sc = p.scale;
-  uint4 o;
-  o.x = pack_bf16x2(a.x * sc, a.y * sc);
-  o.y = pack_bf16x2(a.z * sc, a.w * sc);
-  o.z = pack_bf16x2(c.x * sc, c.y * sc);
-  o.w = pack_bf16x2(c.z * sc, c.w * sc);
-  *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(tok) * p.H + h) * D + 8 * k) = o;
+  for (int e = threadIdx.x; e < 32 * CPR; e += 256) {
+    const int r = e / CPR, c = e % CPR;
+    if (r0 + r >= R) continue;
+    const float4 a = tile[r][2 * c], b = tile[r][2 * c + 1];
+    uint4 o;
+    o.x = pack_bf16x2(a.x * sc, a.y * sc);
+    o.y = pack_bf16x2(a.z * sc, a.w * sc);
+    o.z = pack_bf16x2(b.x * sc, b.y * sc);
+    o.w = pack_bf16x2(b.z * sc, b.w * sc);
+    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(tok0 + r) * p.H + h) * D +
+                              8 * c) = o;
+  }
 }
 
 // ------------------------------------------------------------------ main kernel
