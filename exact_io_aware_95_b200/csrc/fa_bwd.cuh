@@ -42,7 +42,10 @@
 //   warp  12    TMA producer: K_j, V_j once; Q_i and dO_i into a 2-stage ring
 //   warp  13    tensor-memory allocator and the single MMA-issuing thread
 //   warps 14-15 idle
-// Registers (launch 128 each): P/dS warpgroups 152, drain 104, producer/MMA 104.
+// Registers (launch 128 each): P/dS warpgroups 120, drain 168 (it holds a whole
+// 128-column dQ row), producer/MMA 104 (its MMA issue loops stay unrolled over
+// precomputed descriptors: the single issuing thread must keep the tensor
+// pipe fed).
 #pragma once
 #include "sm100_ptx.cuh"
 
@@ -222,7 +225,7 @@ struct BwdCfg {
   static constexpr int LAUNCH_REGS = 128;  // 65536 / 512
   // setmaxnreg split per warpgroup: P/dS (two warpgroups), dQ drain,
   // producer/MMA.  The shares add up to the launch allocation exactly.
-  static constexpr int REGS_PDS = 152, REGS_DRAIN = 104, REGS_PRODUCER = 104;
+  static constexpr int REGS_PDS = 120, REGS_DRAIN = 168, REGS_PRODUCER = 104;
   static_assert(2 * REGS_PDS + REGS_DRAIN + REGS_PRODUCER == 4 * LAUNCH_REGS, "register split");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
 };
@@ -304,7 +307,7 @@ __global__ void __launch_bounds__(512, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 12) {
-    regs_dec<C::REGS_PRODUCER>();
+    regs_set<C::REGS_PRODUCER, C::LAUNCH_REGS>();
   }
   if (warp == 12) {
     // ------------------------------------------------------------ producer
@@ -448,7 +451,7 @@ __global__ void __launch_bounds__(512, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ P^T and dS^T
-    regs_inc<C::REGS_PDS>();
+    regs_set<C::REGS_PDS, C::LAUNCH_REGS>();
     const int w = warp >> 2;          // this warpgroup's query columns: 64w .. 64w+63
     const int t = threadIdx.x & 127;  // key row within the tile == tensor-memory lane
     const int key = k0 + t;
@@ -590,7 +593,7 @@ __global__ void __launch_bounds__(512, 1)
     }
   } else if (warp < 12) {
     // ------------------------------------------------------------ dQ_i drain
-    regs_dec<C::REGS_DRAIN>();
+    regs_set<C::REGS_DRAIN, C::LAUNCH_REGS>();
     if constexpr (DQ) {
       const int t = threadIdx.x - 256;  // query row within the tile == tensor-memory lane
       const uint32_t lane_base = tmem + (static_cast<uint32_t>((warp & 3) * 32) << 16);
@@ -605,28 +608,25 @@ __global__ void __launch_bounds__(512, 1)
         const int64_t R = VARLEN ? p.total : p.N;
         const int64_t r = static_cast<int64_t>(VARLEN ? tok0 : 0) + q;
         float4* acc4 = reinterpret_cast<float4*>(p.dq_acc);
-        // 64 columns at a time; the tile's columns are released once the last
-        // load has landed (the atomics then run from registers)
-#pragma unroll 1
-        for (int cg = 0; cg < D / 32; cg += 2) {
-          uint32_t a[2][32];
-          tmem_ld32(lane_base + C::TM_DQ + 32 * cg, a[0]);
-          tmem_ld32(lane_base + C::TM_DQ + 32 * (cg + 1), a[1]);
-          tmem_wait_ld(a[0]);
-          tmem_wait_ld(a[1]);
-          if (cg + 2 >= D / 32) {
-            tc_fence_before();
-            mbar_arrive(bar(C::BAR_DQ_EMPTY));
-          }
-          if (q < L) {
+        // The whole dQ_i row is loaded first and its tensor-memory columns are
+        // released at once (at d = 128 dP^T(i+1) reuses them); the atomics
+        // then run from registers.  Issuing atomics stalls once the memory
+        // pipeline backs up, so none may stand between dQ_i and dP^T(i+1).
+        uint32_t a[D / 32][32];
 #pragma unroll
-            for (int e = 0; e < 2; ++e)
+        for (int cg = 0; cg < D / 32; ++cg) tmem_ld32(lane_base + C::TM_DQ + 32 * cg, a[cg]);
 #pragma unroll
-              for (int u = 0; u < 8; ++u)
-                atomicAdd(acc4 + dq_acc_index4(bh_, 8 * (cg + e) + u, r, R, D),
-                          make_float4(__uint_as_float(a[e][4 * u]), __uint_as_float(a[e][4 * u + 1]),
-                                      __uint_as_float(a[e][4 * u + 2]), __uint_as_float(a[e][4 * u + 3])));
-          }
+        for (int cg = 0; cg < D / 32; ++cg) tmem_wait_ld(a[cg]);
+        tc_fence_before();
+        mbar_arrive(bar(C::BAR_DQ_EMPTY));
+        if (q < L) {
+#pragma unroll
+          for (int cg = 0; cg < D / 32; ++cg)
+#pragma unroll
+            for (int u = 0; u < 8; ++u)
+              atomicAdd(acc4 + dq_acc_index4(bh_, 8 * cg + u, r, R, D),
+                        make_float4(__uint_as_float(a[cg][4 * u]), __uint_as_float(a[cg][4 * u + 1]),
+                                    __uint_as_float(a[cg][4 * u + 2]), __uint_as_float(a[cg][4 * u + 3])));
         }
       }
     }

@@ -197,7 +197,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
-    regs_dec<104>();
+    regs_set<104, kLaunchRegs>();
   }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -385,7 +385,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
-    regs_inc<200>();
+    regs_set<200, kLaunchRegs>();
     const int k = warp >> 2;
     const int t = threadIdx.x & 127;  // row within the query tile == tensor-memory lane
     const int wq = warp & 3;          // this warp's 32-row quarter

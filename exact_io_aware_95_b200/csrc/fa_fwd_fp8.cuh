@@ -166,7 +166,7 @@ __global__ void __launch_bounds__(384, 1)
   tc_fence_after();
   const uint32_t tmem = *tmem_slot;
   if (warp >= 8) {
-    regs_dec<72>();
+    regs_set<72, kLaunchRegs>();
   }
   if (warp == 8) {
     // ------------------------------------------------------------ producer
@@ -293,7 +293,7 @@ __global__ void __launch_bounds__(384, 1)
     __syncwarp();
   } else if (warp < 8) {
     // ------------------------------------------------------------ softmax / epilogue
-    regs_inc<216>();
+    regs_set<216, kLaunchRegs>();
     const int k = warp >> 2;
     const int t = threadIdx.x & 127;  // row within the query tile == tensor-memory lane
     const int nk = ntile[k];

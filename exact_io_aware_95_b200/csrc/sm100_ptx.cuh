@@ -313,6 +313,18 @@ template <int N>
 __device__ __forceinline__ void regs_dec() {
   asm volatile("setmaxnreg.dec.sync.aligned.u32 %0;" ::"n"(N));
 }
+// Move this warpgroup's register share from the launch allocation LAUNCH to
+// N: setmaxnreg.inc may only raise and setmaxnreg.dec only lower the count,
+// so the direction is chosen here at compile time (nothing when N == LAUNCH).
+template <int N, int LAUNCH>
+__device__ __forceinline__ void regs_set() {
+  static_assert(N % 8 == 0 && N >= 24 && N <= 256, "setmaxnreg count");
+  if constexpr (N > LAUNCH) {
+    regs_inc<N>();
+  } else if constexpr (N < LAUNCH) {
+    regs_dec<N>();
+  }
+}
 }  // namespace fa
 
 namespace fa {
