@@ -462,20 +462,21 @@ __global__ void __launch_bounds__(512, 1)
     const float c = p.scale_log2;
     constexpr float kLog2e = 1.4426950408889634f;
     bool ok = true;
-    // LSE (base 2) and D of this warpgroup's query columns: thread t < 64
+    // -LSE (base 2) and D of this warpgroup's query columns: thread t < 64
     // fetches column 64w + t of the tile starting at q0.  Rows past the
-    // sequence get LSE = +inf so their P is exactly 0.
+    // sequence get -LSE = -inf so their P is exactly 0.
     auto fetch = [&](int q0, float& lv, float& dv) {
       const int q = q0 + 64 * w + t;
-      lv = INFINITY;
+      lv = -INFINITY;
       dv = 0.f;
       if (t < 64 && q < L) {
         const size_t li = VARLEN ? (static_cast<size_t>(h) * p.total + tok0 + q)
                                  : ((static_cast<size_t>(b) * p.H + h) * p.N + q);
-        lv = p.lse[li] * kLog2e;
+        lv = -p.lse[li] * kLog2e;
         dv = p.dvec[li];
       }
     };
+    const uint64_t c2 = f2_pack(c, c);
     float lv_next, dv_next;
     fetch(128 * i_begin, lv_next, dv_next);
     for (int it = 0; it < niter; ++it) {
@@ -505,12 +506,14 @@ __global__ void __launch_bounds__(512, 1)
         tmem_wait_ld(s);
 #pragma unroll
         for (int m = 0; m < 8; ++m) {
-          const float4 l4 = sLSE4[8 * cc + m];
+          const float4 l4 = sLSE4[8 * cc + m];  // -LSE log2(e) of 4 query columns
           const int qa = 32 * cc + 4 * m;
-          float p0 = ex2(fmaf(__uint_as_float(s[4 * m + 0]), c, -l4.x));
-          float p1 = ex2(fmaf(__uint_as_float(s[4 * m + 1]), c, -l4.y));
-          float p2 = ex2(fmaf(__uint_as_float(s[4 * m + 2]), c, -l4.z));
-          float p3 = ex2(fmaf(__uint_as_float(s[4 * m + 3]), c, -l4.w));
+          float x0, x1, x2, x3;
+          f2_unpack(ffma2(f2_pack(__uint_as_float(s[4 * m + 0]), __uint_as_float(s[4 * m + 1])), c2,
+                          f2_pack(l4.x, l4.y)), x0, x1);
+          f2_unpack(ffma2(f2_pack(__uint_as_float(s[4 * m + 2]), __uint_as_float(s[4 * m + 3])), c2,
+                          f2_pack(l4.z, l4.w)), x2, x3);
+          float p0 = ex2(x0), p1 = ex2(x1), p2 = ex2(x2), p3 = ex2(x3);
           if (diag) {
             if (t > qa) p0 = 0.f;
             if (t > qa + 1) p1 = 0.f;
@@ -550,10 +553,13 @@ __global__ void __launch_bounds__(512, 1)
         for (int m = 0; m < 8; ++m) {
           const float4 d4 = sDv4[8 * cc + m];
           const uint32_t a0 = pk[hc][2 * m], a1 = pk[hc][2 * m + 1];
-          const float d0 = bf16lo_to_f32(a0) * (__uint_as_float(dp[4 * m + 0]) - d4.x);
-          const float d1 = bf16hi_to_f32(a0) * (__uint_as_float(dp[4 * m + 1]) - d4.y);
-          const float d2 = bf16lo_to_f32(a1) * (__uint_as_float(dp[4 * m + 2]) - d4.z);
-          const float d3 = bf16hi_to_f32(a1) * (__uint_as_float(dp[4 * m + 3]) - d4.w);
+          float d0, d1, d2, d3;
+          f2_unpack(fmul2(f2_pack(bf16lo_to_f32(a0), bf16hi_to_f32(a0)),
+                          fsub2(f2_pack(__uint_as_float(dp[4 * m + 0]), __uint_as_float(dp[4 * m + 1])),
+                                f2_pack(d4.x, d4.y))), d0, d1);
+          f2_unpack(fmul2(f2_pack(bf16lo_to_f32(a1), bf16hi_to_f32(a1)),
+                          fsub2(f2_pack(__uint_as_float(dp[4 * m + 2]), __uint_as_float(dp[4 * m + 3])),
+                                f2_pack(d4.z, d4.w))), d2, d3);
           wv[2 * m] = pack_bf16x2(d0, d1);
           wv[2 * m + 1] = pack_bf16x2(d2, d3);
         }
