@@ -96,16 +96,27 @@ def test_matches_oracle_within_the_derived_bound(N, causal):
 
 
 @pytest.mark.gpu
-def test_bench_shape_sampled_heads():
-    """B4 H16 N4096 d128 causal with Q, K doubled before quantization."""
-    x8, sc = make_fp8_dense(4, 4096, 16, 128, seed=0, qk_scale_factor=2.0)
+def test_bench_shape_every_head():
+    """B4 H16 N4096 d128 causal with Q, K doubled before quantization: every
+    output element written (NaN-prefilled buffers come back finite) and every
+    (b, h) head within its bound."""
+    from concurrent.futures import ThreadPoolExecutor
+
+    from tests.common import oracle_workers
+    B, N, H, d = 4, 4096, 16, 128
+    x8, sc = make_fp8_dense(B, N, H, d, seed=0, qk_scale_factor=2.0)
     g = {n: t.cuda() for n, t in x8.items()}
-    scale = 1 / math.sqrt(128)
-    o, lse = fa.fwd_fp8(g["q"], g["k"], g["v"], sc["q"], sc["k"], sc["v"], causal=True, scale=scale)
+    scale = 1 / math.sqrt(d)
+    o = torch.full((B, N, H, d), float("nan"), dtype=torch.bfloat16, device="cuda")
+    lse = torch.full((B, H, N), float("nan"), dtype=torch.float32, device="cuda")
+    fa.fwd_fp8(g["q"], g["k"], g["v"], sc["q"], sc["k"], sc["v"], causal=True, scale=scale, out=o, lse=lse)
     fa.check_device_error()
-    for b, h in ((0, 0), (3, 15), (2, 7)):
-        q, k, v = (x8[n][b:b + 1, :, h:h + 1].to(torch.float64).numpy() * sc[n] for n in ("q", "k", "v"))
-        _check_head(q, k, v, o[b:b + 1, :, h:h + 1], lse[b:b + 1, h:h + 1], 0, 0, scale, True)
+    assert torch.isfinite(o).all() and torch.isfinite(lse).all()
+    q, k, v = (_deq(x8[n], sc[n]) for n in ("q", "k", "v"))
+    o, lse = o.cpu(), lse.cpu()
+    pairs = [(b, h) for b in range(B) for h in range(H)]
+    with ThreadPoolExecutor(oracle_workers(len(pairs), 10.0 * N * N * 8)) as ex:
+        list(ex.map(lambda bh: _check_head(q, k, v, o, lse, bh[0], bh[1], scale, True), pairs))
 
 
 @pytest.mark.gpu
