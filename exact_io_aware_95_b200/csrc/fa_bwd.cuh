@@ -157,9 +157,12 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams 
   const int64_t r0 = (blockIdx.x % nblk) * 32;
   const int lane = threadIdx.x & 31, w = threadIdx.x >> 5;
   const float4* acc = reinterpret_cast<const float4*>(p.dq_acc);
+  // streaming (evict-first) loads and stores: the accumulator is dead after
+  // this read and dQ is not read again here, so neither should push out of
+  // L2 the Q, K, V lines the next forward pass reads
 #pragma unroll
   for (int g = w; g < G; g += 8)
-    if (r0 + lane < R) tile[lane][g] = acc[dq_acc_index4(bh, g, r0 + lane, R, D)];
+    if (r0 + lane < R) tile[lane][g] = __ldcs(acc + dq_acc_index4(bh, g, r0 + lane, R, D));
   __syncthreads();
   int h;
   int64_t tok0;
@@ -181,8 +184,8 @@ __global__ void __launch_bounds__(256) fa_bwd_dq_convert_kernel(const BwdParams 
     o.y = pack_bf16x2(a.z * sc, a.w * sc);
     o.z = pack_bf16x2(b.x * sc, b.y * sc);
     o.w = pack_bf16x2(b.z * sc, b.w * sc);
-    *reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(tok0 + r) * p.H + h) * D +
-                              8 * c) = o;
+    __stcs(reinterpret_cast<uint4*>(reinterpret_cast<__nv_bfloat16*>(p.dq) + (static_cast<size_t>(tok0 + r) * p.H + h) * D +
+                                    8 * c), o);
   }
 }
 
