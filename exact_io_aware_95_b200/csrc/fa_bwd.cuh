@@ -231,6 +231,14 @@ struct BwdCfg {
   static constexpr int REGS_PDS = 120, REGS_DRAIN = 168, REGS_PRODUCER = 104;
   static_assert(2 * REGS_PDS + REGS_DRAIN + REGS_PRODUCER == 4 * LAUNCH_REGS, "register split");
   static_assert(SMEM_BYTES <= 232448, "shared memory budget");
+  // The dQ drain pauses this many cycles after every second vector atomic.
+  // Issued back to back, one tile's 4,096 atomics back up the SM's memory
+  // instruction path for about 3,000 cycles, and the MMA warp's tcgen05.mma
+  // and the P/dS warps' shared- and tensor-memory instructions wait behind
+  // them: in clock traces the first dV products of a tile then issue at
+  // ~450 cycles each instead of ~65.  Paced, the atomics still finish well
+  // inside one query tile.
+  static constexpr int DQ_ATOMIC_PAUSE = 60;
 };
 
 // DQ: also form dQ_i = dS K_j per tile and add it into the fp32 accumulator
@@ -632,10 +640,16 @@ __global__ void __launch_bounds__(512, 1)
 #pragma unroll
           for (int cg = 0; cg < D / 32; ++cg)
 #pragma unroll
-            for (int u = 0; u < 8; ++u)
+            for (int u = 0; u < 8; ++u) {
               atomicAdd(acc4 + dq_acc_index4(bh_, 8 * cg + u, r, R, D),
                         make_float4(__uint_as_float(a[cg][4 * u]), __uint_as_float(a[cg][4 * u + 1]),
                                     __uint_as_float(a[cg][4 * u + 2]), __uint_as_float(a[cg][4 * u + 3])));
+              if (u & 1) {
+                const long long t0 = clock64();
+                while (clock64() - t0 < C::DQ_ATOMIC_PAUSE) {
+                }
+              }
+            }
         }
       }
     }
