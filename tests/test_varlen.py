@@ -97,3 +97,33 @@ def test_varlen_total32768_h32_d128_all_sequences():
     assert agg.eo <= O_ATOL and agg.el <= LSE_ATOL, (agg.eo, agg.el)
     assert max(agg.grads()) <= GRAD_RTOL_FRO, agg.grads()
     assert max(agg.worst_head) <= GRAD_RTOL_FRO, agg.worst_head
+
+
+@pytest.mark.parametrize("d", [64, 128])
+@pytest.mark.parametrize("causal", [False, True])
+def test_backward_items_past_sequence_ends(d, causal):
+    """The backward takes (key tile, sequence, head) items from a grid sized by
+    max_seqlen; with max_seqlen well above most lengths most items lie past
+    their sequence's end and must be skipped, while the CTAs that run go on
+    through several real items each.  NaN-prefilled gradients must come back
+    finite, and every sequence and head must match the oracle."""
+    lens = [3, 130, 1, 256, 257, 40, 900, 17, 128, 1100, 5, 384]
+    H = 5
+    x = make_varlen(lens, H, d, seed=12)
+    scale = scale_of(d)
+    cu = x["cu_seqlens"].cuda()
+    g = {k: x[k].cuda() for k in ("q", "k", "v", "do")}
+    mx = 2048  # an upper bound, not the true maximum (1100): extra empty key tiles
+    o, lse = fa.varlen_fwd(g["q"], g["k"], g["v"], cu, mx, causal=causal)
+    dq, dk, dv = nan_like(g["q"]), nan_like(g["k"]), nan_like(g["v"])
+    fa.varlen_bwd(g["q"], g["k"], g["v"], o, lse, g["do"], cu, mx, causal=causal, dq=dq, dk=dk, dv=dv)
+    fa.check_device_error()
+    for t in (dq, dk, dv):
+        assert torch.isfinite(t).all()
+    a = [f64(x[n]) for n in ("q", "k", "v", "do")]
+    G = oracle.attn_varlen_bwd_ref(*a, x["cu_seqlens"].numpy(), scale, causal)
+    cu_h = x["cu_seqlens"].tolist()
+    for s in range(len(lens)):
+        r = slice(cu_h[s], cu_h[s + 1])
+        eg = [rel_fro(f64(t)[r], ref[r]) for t, ref in zip((dq, dk, dv), G)]
+        assert max(eg) <= GRAD_RTOL_FRO, (s, lens[s], eg)
