@@ -324,7 +324,7 @@ fa_status launch_bwd(int dev, const CUtensorMap& mq, const CUtensorMap& mk, cons
     fa::fa_bwd_preprocess_kernel<D><<<preprocess_blocks(dev), 256, 0, s>>>(p);
     if ((st = launch_status(s)) != FA_OK) return st;
   }
-  // 2) fused recompute + dK, dV, dQ accumulation, one CTA per 128-key tile
+  // 2) fused recompute + dK, dV, dQ accumulation: one work item per 128-key tile, taken by persistent CTAs
   {
     const int64_t grid = static_cast<int64_t>(p.nkvtiles) * p.B * p.H;
     if (grid > 0x7fffffff) return FA_ERR_INVALID_ARG;

@@ -10,9 +10,9 @@
 //   1. preprocess   D_i = sum_c dO_ic O_ic (fp32), and the fp32 dQ accumulator
 //                   is zeroed.  D_i equals P_i . dP_i, the row term of the
 //                   softmax Jacobian product.
-//   2. main         one CTA per (128-key tile j, batch entry or sequence, head);
-//                   K_j and V_j stay in shared memory while the CTA loops over
-//                   the query tiles i that can see them:
+//   2. main         one work item per (128-key tile j, sequence or batch entry,
+//                   head), taken by persistent CTAs; K_j, V_j stay in shared
+//                   memory while the CTA loops over the query tiles i they see:
 //                     S^T  = K_j Q_i^T                 (tcgen05, tensor memory)
 //                     P^T  = exp2(S^T c - LSE_i log2 e) -> bf16 in tensor memory
 //                     dP^T = V_j dO_i^T                (tcgen05)
